@@ -1,0 +1,540 @@
+// C ABI of libhardkv.so: argument validation, workspace layout, TMA descriptors and
+// kernel launches for the HARD-KV decode step. No allocation, no synchronisation.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "k_attend.cuh"
+#include "k_score.cuh"
+#include "k_select.cuh"
+#include "k_state.cuh"
+
+using namespace hardkv;
+
+namespace {
+
+thread_local char g_err[256] = "no error";
+
+int cuda_fail(cudaError_t e, const char *what) {
+  snprintf(g_err, sizeof(g_err), "CUDA error in %s: %s (%s)", what, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return HARDKV_ECUDA;
+}
+
+#define HKV_CHECK_LAUNCH(what)                   \
+  do {                                           \
+    cudaError_t e_ = cudaGetLastError();         \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+#define HKV_TRY(expr)            \
+  do {                           \
+    int r_ = (expr);             \
+    if (r_ != HARDKV_OK) return r_; \
+  } while (0)
+
+constexpr int kMinAttendCtas = 444;  // 3 resident attend CTAs x 148 SMs on B200
+constexpr size_t kMaxSmem = 227 * 1024;
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+size_t elem_size(const hardkv_desc *d) { return d->dtype == HARDKV_BF16 ? 2 : 4; }
+
+int validate_desc(const hardkv_desc *d) {
+  if (!d) return HARDKV_EINVAL;
+  if (d->dtype != HARDKV_F32 && d->dtype != HARDKV_BF16) return HARDKV_EDTYPE;
+  if (d->batch < 1 || d->batch > 4096 || d->n_kv_heads < 1 || d->n_q_heads < d->n_kv_heads ||
+      d->n_q_heads % d->n_kv_heads != 0)
+    return HARDKV_EINVAL;
+  if (d->n_q_heads / d->n_kv_heads > 16) return HARDKV_EINVAL;
+  if ((long long)d->batch * d->n_kv_heads > 4096) return HARDKV_EINVAL;
+  if (d->head_dim != 64 && d->head_dim != 128) return HARDKV_EINVAL;
+  if (d->block < 1 || d->block > 64 || d->dense_window < 1 || d->condensed_slots < 1)
+    return HARDKV_EINVAL;
+  if (d->n_sink < 0 || d->n_sink > d->condensed_slots) return HARDKV_EINVAL;
+  if (d->condense_mode != HARDKV_EVICT && d->condense_mode != HARDKV_MERGE) return HARDKV_EINVAL;
+  if (d->sparse_cap < 1) return HARDKV_ECAP;
+  if (d->ring_rows % 64 != 0 || d->ring_rows < d->dense_window + d->block) return HARDKV_ECAP;
+  const long long U = (long long)d->batch * d->n_kv_heads;
+  if (U * d->ring_rows >= (1ll << 31) || U * d->sparse_cap >= (1ll << 31)) return HARDKV_EINVAL;
+  if (d->condense_mode == HARDKV_MERGE &&
+      (d->condensed_slots > 2048 ||
+       condense_smem_floats(d->block, d->head_dim, d->condensed_slots) * 4 > kMaxSmem))
+    return HARDKV_EINVAL;
+  return HARDKV_OK;
+}
+
+Shape make_shape(const hardkv_desc *d) {
+  Shape s;
+  s.B = d->batch;
+  s.Hq = d->n_q_heads;
+  s.H = d->n_kv_heads;
+  s.d = d->head_dim;
+  s.G = d->n_q_heads / d->n_kv_heads;
+  s.blk = d->block;
+  s.W = d->dense_window;
+  s.C = d->condensed_slots;
+  s.n_sink = d->n_sink;
+  s.cap = d->sparse_cap;
+  s.R = d->ring_rows;
+  s.mode = d->condense_mode;
+  s.mask_words = ((d->ring_rows + 1023) / 1024) * 32;
+  s.scale = (float)(1.0 / sqrt((double)d->head_dim));
+  return s;
+}
+
+struct Layout {
+  size_t scores, tile_max, part, pre, st_q, st_k, st_v, st_out, st_tau, total;
+  int tm_stride, P;
+};
+
+Layout layout(const hardkv_desc *d) {
+  Layout L;
+  const size_t U = (size_t)d->batch * d->n_kv_heads, R = d->ring_rows, e = elem_size(d);
+  const int G = d->n_q_heads / d->n_kv_heads;
+  L.tm_stride = kPartsPerTile * (d->ring_rows / kTile + 2);
+  const long long rows_max =
+      (long long)U * (d->sparse_cap + d->dense_window + d->block + d->condensed_slots);
+  const long long minrows = d->dense_window + d->condensed_slots;
+  long long P = (rows_max + 3 * minrows - 1) / (3 * minrows);
+  if (P < kMinAttendCtas) P = kMinAttendCtas;
+  L.P = (int)P;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = round_up(off + bytes, 256);
+    return o;
+  };
+  L.scores = take(U * R * 4);
+  L.tile_max = take(U * (size_t)L.tm_stride * 4);
+  L.part = take((size_t)L.P * kSegMax * G * (d->head_dim + 2) * 4);
+  L.pre = take((U + 1) * 4);
+  L.st_q = take((size_t)d->batch * d->n_q_heads * d->head_dim * e);
+  L.st_k = take(U * d->head_dim * e);
+  L.st_v = take(U * d->head_dim * e);
+  L.st_out = take((size_t)d->batch * d->n_q_heads * d->head_dim * 4);
+  L.st_tau = take(U * 4);
+  L.total = off;
+  return L;
+}
+
+int check_cache(const hardkv_cache *c) {
+  if (!c) return HARDKV_EINVAL;
+  const void *ptrs[] = {c->k_ring, c->v_ring, c->len, c->d_lo, c->s_lo, c->moved, c->k_sp,
+                        c->v_sp, c->sp_idx, c->n_kept, c->k_cd, c->v_cd, c->w_cd, c->status};
+  for (const void *p : ptrs) {
+    if (!p) return HARDKV_EINVAL;
+    if (!aligned16(p)) return HARDKV_EALIGN;
+  }
+  return HARDKV_OK;
+}
+
+int check_ptr(const void *p, bool allow_null = false) {
+  if (!p) return allow_null ? HARDKV_OK : HARDKV_EINVAL;
+  return aligned16(p) ? HARDKV_OK : HARDKV_EALIGN;
+}
+
+int check_common(const hardkv_desc *d, const hardkv_cache *c, const void *ws) {
+  HKV_TRY(validate_desc(d));
+  HKV_TRY(check_cache(c));
+  HKV_TRY(check_ptr(ws));
+  return HARDKV_OK;
+}
+
+Cache make_cache(const hardkv_cache *c) {
+  Cache k;
+  k.k_ring = c->k_ring;
+  k.v_ring = c->v_ring;
+  k.len = c->len;
+  k.d_lo = c->d_lo;
+  k.s_lo = c->s_lo;
+  k.moved = c->moved;
+  k.k_sp = c->k_sp;
+  k.v_sp = c->v_sp;
+  k.sp_idx = c->sp_idx;
+  k.n_kept = c->n_kept;
+  k.k_cd = c->k_cd;
+  k.v_cd = c->v_cd;
+  k.w_cd = c->w_cd;
+  k.status = c->status;
+  return k;
+}
+
+// ---------------------------------------------------------------- device properties
+
+int device_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (device, kernel, size); later
+// calls (for instance during stream capture) only read the cache.
+template <typename K>
+int set_smem(K kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return HARDKV_OK;
+  struct Entry {
+    const void *fn;
+    int dev;
+    size_t bytes;
+  };
+  static Entry done[64];
+  static int n_done = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_done; ++i)
+    if (done[i].fn == (const void *)kernel && done[i].dev == dev && done[i].bytes >= bytes)
+      return HARDKV_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  if (n_done < 64) done[n_done++] = Entry{(const void *)kernel, dev, bytes};
+  return HARDKV_OK;
+}
+
+// ---------------------------------------------------------------- TMA descriptor
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Ring keys as a 2-D bf16 tensor [U*R rows, d channels]; box 64 channels x 64 rows,
+// 128-byte swizzle (matches swz128 in the kernels).
+int make_kmap(CUtensorMap *map, const hardkv_desc *d, void *k_ring) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) {
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled not available from the driver");
+    return HARDKV_ECUDA;
+  }
+  const cuuint64_t rows = (cuuint64_t)d->batch * d->n_kv_heads * d->ring_rows;
+  cuuint64_t dims[2] = {(cuuint64_t)d->head_dim, rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d->head_dim * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, k_ring, dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_err, sizeof(g_err), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return HARDKV_ECUDA;
+  }
+  return HARDKV_OK;
+}
+
+int record(cudaEvent_t *evs, int i, cudaStream_t stream) {
+  if (!evs || !evs[i]) return HARDKV_OK;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaError_t e = cudaStreamIsCapturing(stream, &cs);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+  e = cs == cudaStreamCaptureStatusActive
+          ? cudaEventRecordWithFlags(evs[i], stream, cudaEventRecordExternal)
+          : cudaEventRecord(evs[i], stream);
+  return e == cudaSuccess ? HARDKV_OK : cuda_fail(e, "cudaEventRecord");
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- launches
+
+namespace {
+
+template <typename K>
+int resident_ctas(K kernel, int threads, size_t smem) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess || n < 1)
+    n = 1;
+  return n;
+}
+
+int launch_append(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *k_new,
+                  const void *v_new, cudaStream_t st) {
+  if (d->dtype == HARDKV_BF16)
+    append_kernel<bf16><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const bf16 *>(k_new),
+                                              static_cast<const bf16 *>(v_new));
+  else
+    append_kernel<float><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const float *>(k_new),
+                                               static_cast<const float *>(v_new));
+  HKV_CHECK_LAUNCH("append_kernel");
+  return HARDKV_OK;
+}
+
+int launch_condense(const hardkv_desc *d, const Shape &sh, const Cache &c, cudaStream_t st) {
+  if (d->condense_mode != HARDKV_MERGE) return HARDKV_OK;  // eviction: the append moved s_lo
+  const size_t smem = condense_smem_floats(sh.blk, sh.d, sh.C) * 4;
+  const int U = sh.B * sh.H;
+  if (d->dtype == HARDKV_BF16) {
+    HKV_TRY(set_smem(condense_kernel<bf16>, smem));
+    condense_kernel<bf16><<<U, kCondenseThreads, smem, st>>>(sh, c);
+  } else {
+    HKV_TRY(set_smem(condense_kernel<float>, smem));
+    condense_kernel<float><<<U, kCondenseThreads, smem, st>>>(sh, c);
+  }
+  HKV_CHECK_LAUNCH("condense_kernel");
+  return HARDKV_OK;
+}
+
+template <int D>
+int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
+                     float *scores, float *tm, int tm_stride, int select_mode, cudaStream_t st) {
+  CUtensorMap map;
+  HKV_TRY(make_kmap(&map, d, c.k_ring));
+  const size_t smem = ScoreTma<D>::smem_bytes(sh.B);
+  HKV_TRY(set_smem(score_tma_kernel<D>, smem));
+  static int per_sm = 0;
+  if (!per_sm) per_sm = resident_ctas(score_tma_kernel<D>, ScoreTma<D>::THREADS, smem);
+  const int grid = per_sm * device_sms();
+  score_tma_kernel<D><<<grid, ScoreTma<D>::THREADS, smem, st>>>(
+      sh, c, static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
+  HKV_CHECK_LAUNCH("score_tma_kernel");
+  return HARDKV_OK;
+}
+
+int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, void *ws,
+                 const Layout &L, int select_mode, cudaStream_t st) {
+  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + L.scores);
+  float *tm = reinterpret_cast<float *>(static_cast<char *>(ws) + L.tile_max);
+  if (d->dtype == HARDKV_BF16) {
+    return sh.d == 128 ? launch_score_tma<128>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
+                       : launch_score_tma<64>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
+  }
+  const dim3 grid(sh.R / kTile + 2, sh.B * sh.H);
+  score_f32_kernel<<<grid, 128, (size_t)sh.G * sh.d * 4, st>>>(
+      sh, c, static_cast<const float *>(q), scores, tm, L.tm_stride, select_mode);
+  HKV_CHECK_LAUNCH("score_f32_kernel");
+  return HARDKV_OK;
+}
+
+template <bool WRITE_IDX>
+int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, const float *tau,
+                float p, int select_mode, uint32_t *mask, cudaStream_t st) {
+  const float *scores = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.scores);
+  const float *tm = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.tile_max);
+  topp_kernel<WRITE_IDX><<<sh.B * sh.H, kSelThreads, 0, st>>>(sh, c, scores, tm, L.tm_stride, tau, p,
+                                                             select_mode, mask);
+  HKV_CHECK_LAUNCH("topp_kernel");
+  return HARDKV_OK;
+}
+
+template <typename T, int D>
+int launch_attend_t(const Shape &sh, const Cache &c, const void *q, void *ws, const Layout &L,
+                    int fused, int select_mode, cudaStream_t st) {
+  AttendParams ap;
+  ap.q = q;
+  ap.part = reinterpret_cast<float *>(static_cast<char *>(ws) + L.part);
+  ap.pre_out = reinterpret_cast<int *>(static_cast<char *>(ws) + L.pre);
+  ap.fused = fused;
+  ap.select_mode = select_mode;
+  ap.U = sh.B * sh.H;
+  ap.P = L.P;
+  const size_t smem = AttCfg<T, D>::smem_bytes(ap.U);
+  HKV_TRY(set_smem(attend_kernel<T, D>, smem));
+  attend_kernel<T, D><<<L.P, kAttThreads, smem, st>>>(sh, c, ap);
+  HKV_CHECK_LAUNCH("attend_kernel");
+  return HARDKV_OK;
+}
+
+int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, void *ws,
+                  const Layout &L, int fused, int select_mode, cudaStream_t st) {
+  if (d->dtype == HARDKV_BF16)
+    return sh.d == 128 ? launch_attend_t<bf16, 128>(sh, c, q, ws, L, fused, select_mode, st)
+                       : launch_attend_t<bf16, 64>(sh, c, q, ws, L, fused, select_mode, st);
+  return sh.d == 128 ? launch_attend_t<float, 128>(sh, c, q, ws, L, fused, select_mode, st)
+                     : launch_attend_t<float, 64>(sh, c, q, ws, L, fused, select_mode, st);
+}
+
+int launch_combine(const Shape &sh, void *ws, const Layout &L, float *out, cudaStream_t st) {
+  const float *part = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.part);
+  const int *pre = reinterpret_cast<const int *>(static_cast<char *>(ws) + L.pre);
+  const int U = sh.B * sh.H;
+  if (sh.d == 128)
+    combine_kernel<128><<<U, 128, 0, st>>>(sh, part, pre, U, L.P, out);
+  else
+    combine_kernel<64><<<U, 64, 0, st>>>(sh, part, pre, U, L.P, out);
+  HKV_CHECK_LAUNCH("combine_kernel");
+  return HARDKV_OK;
+}
+
+int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const uint32_t *mask,
+                   int select_mode, cudaStream_t st) {
+  const dim3 grid((sh.R + kSelThreads - 1) / kSelThreads, sh.B * sh.H);
+  if (d->dtype == HARDKV_BF16)
+    compact_kernel<bf16><<<grid, kSelThreads, 0, st>>>(sh, c, mask, select_mode);
+  else
+    compact_kernel<float><<<grid, kSelThreads, 0, st>>>(sh, c, mask, select_mode);
+  HKV_CHECK_LAUNCH("compact_kernel");
+  return HARDKV_OK;
+}
+
+int check_p(float p) { return (p > 0.0f && p <= 1.0f) ? HARDKV_OK : HARDKV_EINVAL; }
+int check_mode(int m) {
+  return (m == HARDKV_SELECT_ALL || m == HARDKV_SELECT_MOVED) ? HARDKV_OK : HARDKV_EINVAL;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- entry points
+
+extern "C" {
+
+size_t hardkv_workspace_bytes(const hardkv_desc *desc) {
+  if (validate_desc(desc) != HARDKV_OK) return 0;
+  return layout(desc).total;
+}
+
+int32_t hardkv_mask_words(const hardkv_desc *desc) {
+  if (validate_desc(desc) != HARDKV_OK) return 0;
+  return make_shape(desc).mask_words;
+}
+
+int hardkv_validate(const hardkv_desc *desc) { return validate_desc(desc); }
+
+int hardkv_append(const hardkv_desc *desc, const hardkv_cache *cache, const void *k_new,
+                  const void *v_new, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(k_new));
+  HKV_TRY(check_ptr(v_new));
+  return launch_append(desc, make_shape(desc), make_cache(cache), k_new, v_new, stream);
+}
+
+int hardkv_condense(const hardkv_desc *desc, const hardkv_cache *cache, void *ws,
+                    cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  return launch_condense(desc, make_shape(desc), make_cache(cache), stream);
+}
+
+int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
+                                const float *tau, float p, int32_t select_mode, uint32_t *mask,
+                                void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(q));
+  HKV_TRY(check_ptr(tau, true));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_p(p));
+  HKV_TRY(check_mode(select_mode));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(cache);
+  const Layout L = layout(desc);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, stream));
+  return launch_topp<false>(sh, c, ws, L, tau, p, select_mode, mask, stream);
+}
+
+int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache, const uint32_t *mask,
+                      int32_t select_mode, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_mode(select_mode));
+  return launch_compact(desc, make_shape(desc), make_cache(cache), mask, select_mode, stream);
+}
+
+int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
+                       float *out, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(q));
+  HKV_TRY(check_ptr(out));
+  const Shape sh = make_shape(desc);
+  const Layout L = layout(desc);
+  HKV_TRY(launch_attend(desc, sh, make_cache(cache), q, ws, L, 0, HARDKV_SELECT_ALL, stream));
+  return launch_combine(sh, ws, L, out, stream);
+}
+
+int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
+                       const hardkv_step_args *a, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  if (!a) return HARDKV_EINVAL;
+  HKV_TRY(check_ptr(a->q));
+  HKV_TRY(check_ptr(a->k_new));
+  HKV_TRY(check_ptr(a->v_new));
+  HKV_TRY(check_ptr(a->tau, true));
+  HKV_TRY(check_ptr(a->mask, true));
+  HKV_TRY(check_ptr(a->out));
+  HKV_TRY(check_p(a->p));
+  HKV_TRY(check_mode(a->select_mode));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(cache);
+  const Layout L = layout(desc);
+  cudaEvent_t *ev = a->stage_events;
+  HKV_TRY(record(ev, 0, stream));
+  HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, stream));
+  HKV_TRY(record(ev, 1, stream));
+  HKV_TRY(launch_condense(desc, sh, c, stream));
+  HKV_TRY(record(ev, 2, stream));
+  HKV_TRY(launch_score(desc, sh, c, a->q, ws, L, a->select_mode, stream));
+  HKV_TRY(record(ev, 3, stream));
+  HKV_TRY(launch_topp<true>(sh, c, ws, L, a->tau, a->p, a->select_mode, a->mask, stream));
+  HKV_TRY(record(ev, 4, stream));
+  HKV_TRY(launch_attend(desc, sh, c, a->q, ws, L, 1, a->select_mode, stream));
+  HKV_TRY(record(ev, 5, stream));
+  HKV_TRY(launch_combine(sh, ws, L, a->out, stream));
+  return record(ev, 6, stream);
+}
+
+int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
+                            const hardkv_step_args *h, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  if (!h || !h->q || !h->k_new || !h->v_new || !h->out) return HARDKV_EINVAL;
+  const Layout L = layout(desc);
+  const size_t e = elem_size(desc);
+  const size_t U = (size_t)desc->batch * desc->n_kv_heads;
+  const size_t nq = (size_t)desc->batch * desc->n_q_heads * desc->head_dim;
+  char *w = static_cast<char *>(ws);
+  hardkv_step_args dv = *h;
+  dv.q = w + L.st_q;
+  dv.k_new = w + L.st_k;
+  dv.v_new = w + L.st_v;
+  dv.out = reinterpret_cast<float *>(w + L.st_out);
+  dv.tau = h->tau ? reinterpret_cast<const float *>(w + L.st_tau) : nullptr;
+  cudaError_t r;
+  if ((r = cudaMemcpyAsync(w + L.st_q, h->q, nq * e, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      (r = cudaMemcpyAsync(w + L.st_k, h->k_new, U * desc->head_dim * e, cudaMemcpyHostToDevice,
+                           stream)) != cudaSuccess ||
+      (r = cudaMemcpyAsync(w + L.st_v, h->v_new, U * desc->head_dim * e, cudaMemcpyHostToDevice,
+                           stream)) != cudaSuccess)
+    return cuda_fail(r, "cudaMemcpyAsync H2D");
+  if (h->tau && (r = cudaMemcpyAsync(w + L.st_tau, h->tau, U * 4, cudaMemcpyHostToDevice, stream)) !=
+                    cudaSuccess)
+    return cuda_fail(r, "cudaMemcpyAsync H2D");
+  HKV_TRY(hardkv_decode_step(desc, cache, &dv, ws, stream));
+  if ((r = cudaMemcpyAsync(h->out, w + L.st_out, nq * 4, cudaMemcpyDeviceToHost, stream)) !=
+      cudaSuccess)
+    return cuda_fail(r, "cudaMemcpyAsync D2H");
+  return HARDKV_OK;
+}
+
+const char *hardkv_strerror(int code) {
+  switch (code) {
+    case HARDKV_OK: return "success";
+    case HARDKV_EINVAL: return "invalid argument (descriptor field, NULL pointer, p or select mode)";
+    case HARDKV_EALIGN: return "pointer not 16-byte aligned";
+    case HARDKV_EDTYPE: return "unsupported dtype";
+    case HARDKV_ECAP: return "capacity rule broken (sparse_cap < 1, ring_rows too small or not a multiple of 64)";
+    case HARDKV_ECUDA: return g_err;
+    default: return "unknown hardkv error code";
+  }
+}
+
+}  // extern "C"

@@ -1,0 +1,241 @@
+// Stage 2a: importance score s_j = max_{g in group(h)} (q_g . k_j) / sqrt(d) over the
+// Sparse candidates (HARD-KV technical summary sec. 2.B: "max-pooled logits").
+//
+// bf16 path: a persistent kernel streams 64-row key tiles of every selected unit's
+// Sparse range with TMA (2-D tensor map over the ring, 128-byte swizzle) into a
+// multi-stage mbarrier pipeline; four consumer warps each take 16 rows of a tile and
+// compute the (query x key) logits with mma.sync m16n8k16 (queries in M, padded to
+// 16; keys in N), then max-pool over the real queries. Work is split evenly over all
+// tiles of all units, so ragged sequence lengths stay balanced.
+#pragma once
+#include "common.cuh"
+
+namespace hardkv {
+
+constexpr int kTile = 64;         // key rows per tile (ring rows are 64-aligned)
+constexpr int kPartsPerTile = 4;  // per-warp partial maxima per tile
+
+template <int D>
+struct ScoreTma {
+  static constexpr int BOXES = D / 64;           // 64-channel TMA boxes per tile
+  static constexpr int BOX_BYTES = kTile * 128;  // 64 rows x 128 bytes
+  static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
+  static constexpr int STAGES = D == 128 ? 6 : 10;
+  static constexpr int CONSUMER_WARPS = 4;
+  static constexpr int THREADS = 32 * (CONSUMER_WARPS + 1);
+  static size_t smem_bytes(int B) {
+    return (size_t)STAGES * TILE_BYTES + 1024 + 2 * STAGES * 8 + 16 + (size_t)(3 * B + 1) * 4;
+  }
+};
+
+// Tiles of sequence b: the 64-aligned position windows meeting [s_lo, d_lo).
+struct TileSpan {
+  int first, n;
+};
+__device__ __forceinline__ TileSpan tile_span(const Bounds &bd) {
+  TileSpan t{0, 0};
+  if (bd.ok && bd.d_lo > bd.s_lo) {
+    t.first = bd.s_lo / kTile;
+    t.n = (bd.d_lo - 1) / kTile - t.first + 1;
+  }
+  return t;
+}
+
+// Loads query fragments (A operand, queries in M) of unit (b,h) for all k-steps.
+template <int D>
+__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[D / 16][4], const bf16 *q, int b,
+                                             int h, const Shape &sh, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const bf16 *q0 = q + ((size_t)b * sh.Hq + (size_t)h * sh.G) * D;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int qi = g + ((r & 1) << 3);
+      const int ch = kk * 16 + ((r >> 1) << 3) + 2 * t;
+      qa[kk][r] = qi < sh.G ? *reinterpret_cast<const uint32_t *>(q0 + (size_t)qi * D + ch) : 0u;
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(ScoreTma<D>::THREADS)
+    score_tma_kernel(Shape sh, Cache c, const bf16 *__restrict__ q, float *__restrict__ scores,
+                     float *__restrict__ tile_max, int tm_stride, int select_mode,
+                     const __grid_constant__ CUtensorMap kmap) {
+  using Cfg = ScoreTma<D>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~uintptr_t(1023));
+  uint64_t *full = reinterpret_cast<uint64_t *>(tiles + Cfg::STAGES * Cfg::TILE_BYTES);
+  uint64_t *empty = full + Cfg::STAGES;
+  int *abort_flag = reinterpret_cast<int *>(empty + Cfg::STAGES);
+  int *pre = abort_flag + 4;        // [B+1] tile prefix
+  int *first = pre + sh.B + 1;      // [B]
+  int *ntile = first + sh.B;        // [B]
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], Cfg::CONSUMER_WARPS);
+    }
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == Cfg::CONSUMER_WARPS && lane == 0) tma_prefetch_desc(&kmap);
+  if (warp == 0) {  // per-sequence tile spans and their prefix over (b, h)
+    int carry = 0;
+    for (int b0 = 0; b0 < sh.B; b0 += 32) {
+      const int b = b0 + lane;
+      int v = 0;
+      if (b < sh.B) {
+        TileSpan ts{0, 0};
+        if (unit_active(select_mode, c.moved, b)) ts = tile_span(load_bounds(c, b, sh.R));
+        first[b] = ts.first;
+        ntile[b] = ts.n;
+        v = ts.n * sh.H;
+      }
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (b < sh.B) pre[b + 1] = carry + incl;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) pre[0] = 0;
+  }
+  __syncthreads();
+
+  const long long total = pre[sh.B];
+  const long long g0 = total * blockIdx.x / gridDim.x;
+  const long long g1 = total * (blockIdx.x + 1) / gridDim.x;
+  if (g0 >= g1) return;
+
+  if (warp == Cfg::CONSUMER_WARPS) {
+    // ---------------- producer: one thread issues the TMA loads
+    if (lane != 0) return;
+    int b = 0;
+    long long issued = 0;
+    for (long long g = g0; g < g1; ++g, ++issued) {
+      while (g >= pre[b + 1]) ++b;
+      const int idx = (int)(g - pre[b]);
+      const int h = idx / ntile[b], lt = idx % ntile[b];
+      const int u = b * sh.H + h;
+      const int row0 = (int)(((long long)(first[b] + lt) * kTile) % sh.R);
+      const int st = (int)(issued % Cfg::STAGES);
+      const uint32_t par = (uint32_t)((issued / Cfg::STAGES) & 1) ^ 1u;
+      if (*(volatile int *)abort_flag || !mbar_wait(&empty[st], par)) {
+        *(volatile int *)abort_flag = 1;
+        flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
+        break;
+      }
+      mbar_arrive_expect_tx(&full[st], Cfg::TILE_BYTES);
+#pragma unroll
+      for (int bx = 0; bx < Cfg::BOXES; ++bx)
+        tma_load_2d(tiles + st * Cfg::TILE_BYTES + bx * Cfg::BOX_BYTES, &kmap, bx * 64,
+                    u * sh.R + row0, &full[st]);
+    }
+    // drain: the last loads issued must land before the CTA may exit
+    for (long long j = issued > Cfg::STAGES ? issued - Cfg::STAGES : 0; j < issued; ++j)
+      mbar_wait(&full[j % Cfg::STAGES], (uint32_t)((j / Cfg::STAGES) & 1));
+    return;
+  }
+
+  // ---------------- consumers: warp w takes rows [16w, 16w+16) of every tile
+  const int g = lane >> 2, t = lane & 3;
+  uint32_t qa[D / 16][4];
+  int cur_u = -1, b = 0;
+  long long i = 0;
+  for (long long gg = g0; gg < g1; ++gg, ++i) {
+    while (gg >= pre[b + 1]) ++b;
+    const int idx = (int)(gg - pre[b]);
+    const int h = idx / ntile[b], lt = idx % ntile[b];
+    const int u = b * sh.H + h;
+    if (u != cur_u) {
+      load_q_frags<D>(qa, q, b, h, sh, lane);
+      cur_u = u;
+    }
+    const int st = (int)(i % Cfg::STAGES);
+    if (*(volatile int *)abort_flag || !mbar_wait(&full[st], (uint32_t)((i / Cfg::STAGES) & 1))) {
+      *(volatile int *)abort_flag = 1;
+      flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
+      break;
+    }
+    const uint32_t base = smem_u32(tiles + st * Cfg::TILE_BYTES);
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int r = warp * 16 + (lane & 7) + (((lane >> 4) & 1) << 3);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int ch = kk * 16 + (((lane >> 3) & 1) << 3);
+      const uint32_t addr = base + (ch >> 6) * Cfg::BOX_BYTES + swz128(r, (ch & 63) >> 3);
+      uint32_t b0, b1, b2, b3;
+      ldsm_x4(b0, b1, b2, b3, addr);
+      mma_bf16(acc[0], qa[kk], b0, b1);
+      mma_bf16(acc[1], qa[kk], b2, b3);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[st]);
+
+    // max-pool over the real queries (rows g and g+8 of M)
+    const Bounds bd{c.len[b], c.d_lo[b], c.s_lo[b], true};
+    const long long pbase = (long long)(first[b] + lt) * kTile + warp * 16;
+    float tmax = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 2; ++n) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float v = fmaxf(g < sh.G ? acc[n][e] : -INFINITY, g + 8 < sh.G ? acc[n][2 + e] : -INFINITY);
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
+        const long long pos = pbase + n * 8 + 2 * t + e;
+        if (lane < 4 && pos >= bd.s_lo && pos < bd.d_lo) {
+          const float s = v * sh.scale;
+          scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
+          tmax = fmaxf(tmax, s);
+        }
+      }
+    }
+    tmax = warp_max(tmax);
+    if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + warp] = tmax;
+  }
+}
+
+// fp32 keys: one CTA per (tile, unit); 4 warps x 16 rows; lanes split channels.
+__global__ void __launch_bounds__(128)
+    score_f32_kernel(Shape sh, Cache c, const float *__restrict__ q, float *__restrict__ scores,
+                     float *__restrict__ tile_max, int tm_stride, int select_mode) {
+  const int u = blockIdx.y, b = u / sh.H, h = u % sh.H;
+  if (!unit_active(select_mode, c.moved, b)) return;
+  const Bounds bd = load_bounds(c, b, sh.R);
+  const TileSpan ts = tile_span(bd);
+  const int lt = blockIdx.x;
+  if (lt >= ts.n) return;
+  extern __shared__ float qs[];  // [G][d]
+  for (int i = threadIdx.x; i < sh.G * sh.d; i += blockDim.x)
+    qs[i] = q[((size_t)b * sh.Hq + (size_t)h * sh.G) * sh.d + i];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float *kr = static_cast<const float *>(c.k_ring) + (size_t)u * sh.R * sh.d;
+  float tmax = -INFINITY;
+  for (int r = 0; r < 16; ++r) {
+    const long long pos = (long long)(ts.first + lt) * kTile + warp * 16 + r;
+    if (pos < bd.s_lo || pos >= bd.d_lo) continue;
+    const float *krow = kr + (size_t)(pos % sh.R) * sh.d;
+    float best = -INFINITY;
+    for (int gq = 0; gq < sh.G; ++gq) {
+      float a = 0.f;
+      for (int ch = lane; ch < sh.d; ch += 32) a += qs[gq * sh.d + ch] * krow[ch];
+      best = fmaxf(best, warp_sum(a));
+    }
+    const float s = best * sh.scale;
+    if (lane == 0) scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
+    tmax = fmaxf(tmax, s);
+  }
+  if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + warp] = tmax;
+}
+
+}  // namespace hardkv

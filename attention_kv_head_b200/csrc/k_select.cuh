@@ -1,0 +1,368 @@
+// Stage 2b/2c: Logits Calibration + calibrated top-p (HARD-KV technical summary sec.
+// 2.B, sec. 2.A Tier 2) and stage 3, Index Regularization by prefix scan (sec. 2.C
+// Rewrite Cache, Flatten Index to the maximum length).
+//
+// Top-p without a sort: the calibrated mass of candidate j is
+//   m_j = exp((s_j - max s) / tau)      (unnormalised; the threshold is p * sum m)
+// held as 40-bit fixed point so every sum is an exact, order-independent integer.
+// A three-pass radix select (11 + 11 + 10 bits of an order-preserving key of s)
+// finds the key theta of the last kept candidate of the (s desc, position asc) order:
+// the shortest prefix whose mass reaches p * Z or whose length reaches Cap.
+#pragma once
+#include "common.cuh"
+#include "k_score.cuh"
+
+namespace hardkv {
+
+constexpr int kSelThreads = 1024;
+constexpr float kMassScale = 1099511627776.0f;  // 2^40
+
+// Exclusive scan of a 0/1 flag over a 1024-thread block; returns (excl, total).
+// `ws` is 33 ints of shared memory. Contains __syncthreads(); call uniformly.
+__device__ __forceinline__ int2 block_scan_flag(bool f, int *ws) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, f);
+  const int lx = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) ws[warp] = __popc(bal);
+  __syncthreads();
+  if (warp == 0) {
+    const int v = ws[lane];
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    ws[lane] = incl - v;
+    if (lane == 31) ws[32] = incl;
+  }
+  __syncthreads();
+  const int2 r = make_int2(ws[warp] + lx, ws[32]);
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ float block_max(float v, float *ws) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  v = warp_max(v);
+  if (lane == 0) ws[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    float x = lane < (int)(blockDim.x >> 5) ? ws[lane] : -INFINITY;
+    x = warp_max(x);
+    if (lane == 0) ws[32] = x;
+  }
+  __syncthreads();
+  const float r = ws[32];
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long mass_fx(float s, float M, float tau) {
+  return __float2ull_rn(expf((s - M) / tau) * kMassScale);
+}
+
+struct SelShared {
+  uint32_t cnt[2048];
+  unsigned long long mass[2048];
+  unsigned long long wmass[32];
+  uint32_t wcnt[32];
+  int scan[40];
+  float red[40];
+  int sel_bin;
+  uint32_t sel_cnt;
+  unsigned long long sel_mass;
+};
+
+// One CTA per (b,h). Writes the mask (if not NULL) and, with WRITE_IDX, the compact
+// index list sp_idx / n_kept (positions of kept candidates in ascending order).
+template <bool WRITE_IDX>
+__global__ void __launch_bounds__(kSelThreads)
+    topp_kernel(Shape sh, Cache c, const float *__restrict__ scores,
+                const float *__restrict__ tile_max, int tm_stride, const float *__restrict__ tau,
+                float p, int select_mode, uint32_t *__restrict__ mask) {
+  const int u = blockIdx.x, b = u / sh.H;
+  if (!unit_active(select_mode, c.moved, b)) return;
+  __shared__ SelShared S;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Bounds bd = load_bounds(c, b, sh.R);
+  if (!bd.ok && tid == 0) flag(c.status, HARDKV_DEV_BAD_BOUNDS);
+  const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
+  const float *sc = scores + (size_t)u * sh.R;
+  const float tv = tau ? tau[u] : 1.0f;
+
+  // max score from the per-tile partial maxima
+  const TileSpan ts = tile_span(bd);
+  float m = -INFINITY;
+  for (int i = tid; i < ts.n * kPartsPerTile; i += kSelThreads)
+    m = fmaxf(m, tile_max[(size_t)u * tm_stride + i]);
+  const float M = block_max(m, S.red);
+
+  uint32_t prefix = 0, pmask = 0, above_cnt = 0;
+  unsigned long long above_mass = 0, T = ~0ull, mth = 0;
+  uint32_t E = 0;
+  bool keep_all = (L == 0);
+  const uint32_t cap = (uint32_t)sh.cap;
+  for (int pass = 0; pass < 3 && !keep_all; ++pass) {
+    const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    const int nb = pass == 2 ? 1024 : 2048;
+    for (int i = tid; i < nb; i += kSelThreads) {
+      S.cnt[i] = 0;
+      S.mass[i] = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < L; base += kSelThreads) {
+      const int j = base + tid;
+      bool pred = false;
+      float s = 0.f;
+      uint32_t key = 0;
+      if (j < L) {
+        s = sc[j];
+        key = order_key(s);
+        pred = (key & pmask) == prefix;
+      }
+      const unsigned act = __ballot_sync(0xffffffffu, pred);
+      if (pred) {
+        const uint32_t bin = (key >> shift) & (uint32_t)(nb - 1);
+        const unsigned long long mv = mass_fx(s, M, tv);
+        const unsigned peers = __match_any_sync(act, bin);
+        const uint32_t lo = __reduce_add_sync(peers, (uint32_t)(mv & 0xFFFFFull));
+        const uint32_t hi = __reduce_add_sync(peers, (uint32_t)(mv >> 20));
+        if (lane == __ffs(peers) - 1) {
+          atomicAdd(&S.cnt[bin], (uint32_t)__popc(peers));
+          atomicAdd(&S.mass[bin], (unsigned long long)lo + ((unsigned long long)hi << 20));
+        }
+      }
+    }
+    __syncthreads();
+    // suffix sums over bins, highest bin first; thread handles nb/1024 bins
+    const int per = nb / kSelThreads;
+    uint32_t lc = 0;
+    unsigned long long lm = 0;
+    for (int k = 0; k < per; ++k) {
+      const int bin = nb - 1 - (tid * per + k);
+      lc += S.cnt[bin];
+      lm += S.mass[bin];
+    }
+    // block exclusive scan of (lc, lm)
+    uint32_t ic = lc;
+    unsigned long long im = lm;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t yc = __shfl_up_sync(0xffffffffu, ic, o);
+      const unsigned long long ym = __shfl_up_sync(0xffffffffu, im, o);
+      if (lane >= o) {
+        ic += yc;
+        im += ym;
+      }
+    }
+    if (lane == 31) {
+      S.wcnt[warp] = ic;
+      S.wmass[warp] = im;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      uint32_t vc = S.wcnt[lane];
+      unsigned long long vm = S.wmass[lane];
+      uint32_t xc = vc;
+      unsigned long long xm = vm;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t yc = __shfl_up_sync(0xffffffffu, xc, o);
+        const unsigned long long ym = __shfl_up_sync(0xffffffffu, xm, o);
+        if (lane >= o) {
+          xc += yc;
+          xm += ym;
+        }
+      }
+      S.wcnt[lane] = xc - vc;
+      S.wmass[lane] = xm - vm;
+      if (lane == 31 && pass == 0) {
+        // total calibrated mass Z; threshold T = ceil(p Z) (p >= 1 keeps all)
+        const unsigned long long Z = xm;
+        S.sel_mass = p >= 1.0f ? ~0ull
+                               : (unsigned long long)ceil((double)p * (double)Z);
+      }
+      if (lane == 0) S.sel_bin = -1;
+    }
+    __syncthreads();
+    if (pass == 0) T = S.sel_mass;
+    __syncthreads();
+    {
+      uint32_t cc = above_cnt + S.wcnt[warp] + (ic - lc);
+      unsigned long long cm = above_mass + S.wmass[warp] + (im - lm);
+      for (int k = 0; k < per; ++k) {
+        const int bin = nb - 1 - (tid * per + k);
+        const uint32_t nc = cc + S.cnt[bin];
+        const unsigned long long nm = cm + S.mass[bin];
+        const bool crit_above = cm >= T || cc >= cap;
+        const bool crit_incl = nm >= T || nc >= cap;
+        if (crit_incl && !crit_above) {
+          S.sel_bin = bin;
+          S.sel_cnt = cc;
+          S.sel_mass = cm;
+        }
+        cc = nc;
+        cm = nm;
+      }
+    }
+    __syncthreads();
+    const int sb = S.sel_bin;
+    if (sb < 0) {
+      keep_all = true;  // the whole remaining range is needed (only when p >= 1 or L <= Cap)
+    } else {
+      above_cnt = S.sel_cnt;
+      above_mass = S.sel_mass;
+      prefix |= (uint32_t)sb << shift;
+      pmask |= (uint32_t)(nb - 1) << shift;
+      if (pass == 2) {
+        E = S.cnt[sb];
+        mth = E ? S.mass[sb] / E : 0;
+      }
+    }
+    __syncthreads();
+  }
+
+  // number of candidates with key == theta to keep (lowest positions first)
+  uint32_t r = 0, n = (uint32_t)L;
+  bool clamped = false;
+  if (!keep_all) {
+    const unsigned long long need = T > above_mass ? T - above_mass : 0ull;
+    uint32_t r_mass = E;
+    if (T != ~0ull && mth > 0) {
+      const unsigned long long q = (need + mth - 1) / mth;
+      r_mass = q < E ? (uint32_t)q : E;
+    }
+    const uint32_t r_cap = cap - above_cnt;
+    r = min(E, min(r_mass, r_cap));
+    n = above_cnt + r;
+    clamped = (n == cap) && (above_mass + (unsigned long long)r * mth < T);
+  } else if ((uint32_t)L > cap) {
+    n = cap;  // unreachable: the count rule fires first when L > Cap
+  }
+  const bool need_rank = !keep_all && r < E;
+  const uint32_t theta = prefix;
+
+  int run_eq = 0, run_kept = 0;
+  int32_t *idx = WRITE_IDX ? c.sp_idx + (size_t)u * sh.cap : nullptr;
+  for (int base = 0; base < L; base += kSelThreads) {
+    const int j = base + tid;
+    const bool valid = j < L;
+    const uint32_t key = valid ? order_key(sc[j]) : 0u;
+    const bool eq = valid && !keep_all && key == theta;
+    int rank = 0;
+    if (need_rank) {
+      const int2 e = block_scan_flag(eq, S.scan);
+      rank = run_eq + e.x;
+      run_eq += e.y;
+    }
+    const bool kept = valid && (keep_all || key > theta || (eq && (!need_rank || rank < (int)r)));
+    const unsigned word = __ballot_sync(0xffffffffu, kept);
+    if (mask && lane == 0) mask[(size_t)u * sh.mask_words + ((base >> 5) + warp)] = word;
+    if (WRITE_IDX) {
+      const int2 e = block_scan_flag(kept, S.scan);
+      const int slot = run_kept + e.x;
+      if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
+      run_kept += e.y;
+    }
+  }
+  if (mask) {
+    const int w0 = ((L + kSelThreads - 1) / kSelThreads) * (kSelThreads / 32);
+    for (int w = w0 + tid; w < sh.mask_words; w += kSelThreads) mask[(size_t)u * sh.mask_words + w] = 0u;
+  }
+  if (WRITE_IDX) {
+    for (int s = (int)n + tid; s < sh.cap; s += kSelThreads) idx[s] = -1;
+    if (tid == 0) c.n_kept[u] = (int)n;
+  }
+  if (tid == 0) {
+    if (clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
+    atomicAdd(c.status + HARDKV_ST_SELECTIONS, 1u);
+  }
+}
+
+// Standalone Index Regularization from a mask. Grid (chunks of 1024 candidates, U);
+// warp w of chunk k owns mask word 32k + w.
+template <typename T>
+__global__ void __launch_bounds__(kSelThreads)
+    compact_kernel(Shape sh, Cache c, const uint32_t *__restrict__ mask, int select_mode) {
+  const int u = blockIdx.y, b = u / sh.H;
+  if (!unit_active(select_mode, c.moved, b)) return;
+  __shared__ int scan[40];
+  __shared__ int list_slot[kSelThreads];
+  __shared__ int list_pos[kSelThreads];
+  __shared__ unsigned long long red[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const Bounds bd = load_bounds(c, b, sh.R);
+  const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
+  const int nwords = (L + 31) / 32;
+  const int chunk = blockIdx.x;
+  const uint32_t *mw = mask + (size_t)u * sh.mask_words;
+  auto word_at = [&](int w) -> uint32_t {
+    if (w >= nwords) return 0u;
+    const int rem = L - 32 * w;
+    const uint32_t m = rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u);
+    return mw[w] & m;
+  };
+  // kept before this chunk, and in total
+  unsigned long long before = 0, total = 0;
+  for (int w = tid; w < nwords; w += kSelThreads) {
+    const unsigned long long pc = __popc(word_at(w));
+    total += pc;
+    if (w < chunk * 32) before += pc;
+  }
+  const unsigned long long packed = (before << 32) | total;
+  unsigned long long v = packed;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    unsigned long long x = red[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) red[0] = x;
+  }
+  __syncthreads();
+  const unsigned long long agg = red[0];
+  const int n_before = (int)(agg >> 32);
+  const int n_total = (int)(agg & 0xffffffffull);
+  const int n = min(n_total, sh.cap);
+  int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
+  if (chunk == 0) {
+    for (int s = n + tid; s < sh.cap; s += kSelThreads) idx[s] = -1;
+    if (tid == 0) {
+      c.n_kept[u] = n;
+      if (n_total > sh.cap) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
+    }
+  }
+  if (chunk * kSelThreads >= L) return;
+  const uint32_t bits = word_at(chunk * 32 + warp);
+  const bool kept = (bits >> lane) & 1u;
+  const int2 e = block_scan_flag(kept, scan);
+  if (kept) {
+    list_slot[e.x] = n_before + e.x;
+    list_pos[e.x] = bd.s_lo + chunk * kSelThreads + warp * 32 + lane;
+  }
+  __syncthreads();
+  const int cnt = e.y;
+  const int vec = sh.d * (int)sizeof(T) / 16;
+  const T *kr = static_cast<const T *>(c.k_ring) + (size_t)u * sh.R * sh.d;
+  const T *vr = static_cast<const T *>(c.v_ring) + (size_t)u * sh.R * sh.d;
+  T *ks = static_cast<T *>(c.k_sp) + (size_t)u * sh.cap * sh.d;
+  T *vs = static_cast<T *>(c.v_sp) + (size_t)u * sh.cap * sh.d;
+  for (int i = tid; i < cnt * 2 * vec; i += kSelThreads) {
+    const int e2 = i / (2 * vec), kv = (i / vec) & 1, v2 = i % vec;
+    const int slot = list_slot[e2];
+    if (slot >= sh.cap) continue;
+    const int pos = list_pos[e2];
+    const size_t src_row = (size_t)(pos % sh.R) * sh.d, dst_row = (size_t)slot * sh.d;
+    if (kv == 0) {
+      reinterpret_cast<uint4 *>(ks + dst_row)[v2] = reinterpret_cast<const uint4 *>(kr + src_row)[v2];
+      if (v2 == 0) idx[slot] = pos;
+    } else {
+      reinterpret_cast<uint4 *>(vs + dst_row)[v2] = reinterpret_cast<const uint4 *>(vr + src_row)[v2];
+    }
+  }
+}
+
+}  // namespace hardkv

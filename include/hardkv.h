@@ -1,0 +1,220 @@
+/*
+ * hardkv.h — C ABI of the HARD-KV decode-step library (libhardkv.so, sm_100a).
+ *
+ * HARD-KV ("HARD-KV: Head-Adaptive Regularization for Decoding-time KV
+ * Compression", technical summary sec. 2 "Methodology") keeps each attention
+ * layer's KV cache in three tiers per (sequence b, KV head h):
+ *   Dense     positions [d_lo, len)   most recent tokens, contiguous (Tier 1)
+ *   Sparse    positions [s_lo, d_lo)  aged-out tokens; calibrated top-p keeps a
+ *                                     head-adaptive subset (Tier 2)
+ *   Condensed C slots                 oldest tokens, evicted or merged (Tier 3)
+ * and runs every decode step through four stages (sec. 2.A): (1) linear append
+ * to Dense; (2) Logits Calibration + top-p -> selection masks; (3) Index
+ * Regularization: kept rows rewritten into a contiguous fixed-capacity layout
+ * (sec. 2.C Rewrite Cache, Flatten Index to the maximum length); (4) eviction or
+ * weighted merge of the oldest block; then decode attention over the tiers.
+ *
+ * Conventions for every entry point:
+ *  - Pointers marked "device" are CUDA device pointers owned by the caller; the
+ *    library allocates nothing, never synchronises, keeps no state between calls
+ *    and only enqueues work on `stream`. Every entry point can be captured in a
+ *    CUDA graph (shapes come from the descriptor, tier boundaries live on the
+ *    device).
+ *  - Every device pointer must be 16-byte aligned; head_dim * element size is a
+ *    multiple of 16 by construction (head_dim 64 or 128).
+ *  - Element type of K, V, q, k_new, v_new is `desc->dtype` (IEEE float32 or
+ *    bfloat16). Attention output is float32.
+ *  - Layouts are row-major, innermost dimension last:
+ *      ring K/V  [B, H, R, d]   position p of unit (b,h) lives in row p mod R
+ *      compact   [B, H, Cap, d] slots 0..n-1 valid
+ *      condensed [B, H, C, d]   weights [B, H, C] float32 (0 = empty slot)
+ *      q [B, Hq, d]; query head qh belongs to KV head qh / (Hq / H)
+ *  - Return value: HARDKV_OK (0) or a negative HARDKV_E* code. Arguments are
+ *    validated before anything is enqueued; on an error nothing is enqueued.
+ *    HARDKV_ECUDA means a launch failed; hardkv_strerror() then names the CUDA
+ *    error. Anomalies found on the device (inconsistent boundaries, capacity
+ *    clamps, merge near-ties) are recorded in the caller's status words, never
+ *    trapped.
+ */
+#ifndef HARDKV_H
+#define HARDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HARDKV_OK 0
+#define HARDKV_EINVAL (-1)   /* bad descriptor field, NULL pointer or p outside (0,1] */
+#define HARDKV_EALIGN (-2)   /* a pointer is not 16-byte aligned */
+#define HARDKV_EDTYPE (-3)   /* dtype not HARDKV_F32 / HARDKV_BF16 */
+#define HARDKV_ECAP   (-4)   /* capacity rule broken (Cap < 1, R too small, R % 64) */
+#define HARDKV_ECUDA  (-5)   /* a CUDA launch or copy failed */
+
+enum { HARDKV_F32 = 0, HARDKV_BF16 = 1 };
+enum { HARDKV_EVICT = 0, HARDKV_MERGE = 1 };
+/* Which sequences reselect their Sparse subset in a call:
+ * ALL   = every sequence;
+ * MOVED = only sequences whose last hardkv_append moved a block (moved[b] != 0),
+ *         i.e. each sequence reselects once per block of decode steps. */
+enum { HARDKV_SELECT_ALL = 0, HARDKV_SELECT_MOVED = 1 };
+
+/* Device status words (caller-allocated uint32[HARDKV_STATUS_WORDS], zeroed by the
+ * caller when it wants to start counting). */
+#define HARDKV_STATUS_WORDS 8
+enum {
+  HARDKV_ST_FLAGS = 0,      /* OR of HARDKV_DEV_* bits */
+  HARDKV_ST_CLAMPS = 1,     /* selections whose top-p count exceeded Cap */
+  HARDKV_ST_NEAR_TIES = 2,  /* merges whose best two cosines differ by <= 1e-6 */
+  HARDKV_ST_MERGED = 3,     /* tokens merged into the Condensed tier */
+  HARDKV_ST_MOVES = 4,      /* block moves (one per sequence and move) */
+  HARDKV_ST_SELECTIONS = 5  /* (sequence, head) top-p selections performed */
+};
+#define HARDKV_DEV_RING_OVERFLOW 1u  /* append would overwrite a live ring row: skipped */
+#define HARDKV_DEV_BAD_BOUNDS    2u  /* s_lo <= d_lo <= len broken or span > R: unit skipped */
+#define HARDKV_DEV_SEGMENTS      4u  /* attention partition had to drop a segment */
+#define HARDKV_DEV_WAIT_TIMEOUT  8u  /* a pipeline wait hit its iteration limit */
+
+/* Static shape of one attention layer's cascade cache. */
+typedef struct {
+  int32_t batch;            /* B: sequences */
+  int32_t n_q_heads;        /* Hq: query heads; Hq % H == 0, G = Hq / H in 1..16 */
+  int32_t n_kv_heads;       /* H: KV heads */
+  int32_t head_dim;         /* d: 64 or 128 */
+  int32_t block;            /* tokens per block moved between tiers, 1..64 */
+  int32_t dense_window;     /* W: Dense tier holds W .. W+block-1 tokens */
+  int32_t condensed_slots;  /* C: Condensed slots per (b,h), >= 1 (<= 2048 for MERGE) */
+  int32_t n_sink;           /* slots [0, n_sink) are pinned (never merged into) */
+  int32_t sparse_cap;       /* Cap: compact rows per (b,h), >= 1 */
+  int32_t ring_rows;        /* R: raw rows per (b,h); multiple of 64; the live span
+                               [s_lo, len) must stay <= R (R >= Sparse + W + block) */
+  int32_t dtype;            /* HARDKV_F32 or HARDKV_BF16 */
+  int32_t condense_mode;    /* HARDKV_EVICT or HARDKV_MERGE */
+} hardkv_desc;
+
+/* The cache state: all device pointers, caller-owned. */
+typedef struct {
+  void *k_ring, *v_ring;    /* [B,H,R,d] raw rows (Dense + Sparse candidates) */
+  int32_t *len;             /* [B] tokens so far (positions 0..len-1) */
+  int32_t *d_lo;            /* [B] first Dense position */
+  int32_t *s_lo;            /* [B] first Sparse position (positions < s_lo are condensed) */
+  int32_t *moved;           /* [B] 1 if the last append moved a block, else 0 */
+  void *k_sp, *v_sp;        /* [B,H,Cap,d] compact (regularized) kept rows */
+  int32_t *sp_idx;          /* [B,H,Cap] position of each compact slot, -1 = pad */
+  int32_t *n_kept;          /* [B,H] compact slots in use */
+  void *k_cd, *v_cd;        /* [B,H,C,d] Condensed slots */
+  float *w_cd;              /* [B,H,C] Condensed weights (tokens merged in), 0 = empty */
+  uint32_t *status;         /* [HARDKV_STATUS_WORDS] device counters and flags */
+} hardkv_cache;
+
+/* Arguments of one fused decode step. */
+typedef struct {
+  const void *q;            /* [B,Hq,d] this step's queries */
+  const void *k_new;        /* [B,H,d] this step's key */
+  const void *v_new;        /* [B,H,d] this step's value */
+  const float *tau;         /* [B,H] calibration temperatures (device), or NULL = 1 */
+  float p;                  /* top-p mass, 0 < p <= 1 (p = 1 keeps every candidate) */
+  int32_t select_mode;      /* HARDKV_SELECT_ALL or HARDKV_SELECT_MOVED */
+  uint32_t *mask;           /* [B,H,mask_words] selection masks out (device), or NULL */
+  float *out;               /* [B,Hq,d] attention output */
+  cudaEvent_t *stage_events;/* NULL, or HARDKV_STEP_EVENTS events recorded before the
+                               first stage and after each stage (capture-safe) */
+} hardkv_step_args;
+#define HARDKV_STEP_EVENTS 7  /* start, append, condense, score, topp, attend, combine */
+
+/* Bytes of scratch the library needs for this descriptor (caller allocates; the
+ * content need not be initialised and is not read across calls except as noted). */
+size_t hardkv_workspace_bytes(const hardkv_desc *desc);
+
+/* uint32 words per (b,h) in a selection mask: bit j of unit (b,h) = Sparse
+ * candidate j, i.e. position s_lo[b] + j. */
+int32_t hardkv_mask_words(const hardkv_desc *desc);
+
+/* Check a descriptor alone. Returns HARDKV_OK or the error code the entry points
+ * would return. Pure host code: no CUDA call. */
+int hardkv_validate(const hardkv_desc *desc);
+
+/* Stage 1 (sec. 2.A stage (1), "linear append to the Dense cache").
+ * For each sequence b: writes k_new[b,h], v_new[b,h] (device, [B,H,d]) to ring row
+ * len[b] mod R, then len[b] += 1. If now len - d_lo >= W + block, one block moves
+ * Dense->Sparse (d_lo += block) and the oldest Sparse block leaves for the Condensed
+ * tier (s_lo += block); moved[b] records whether that happened. If the write would
+ * overrun the ring (len - s_lo >= R) the sequence is skipped and
+ * HARDKV_DEV_RING_OVERFLOW is raised. */
+int hardkv_append(const hardkv_desc *desc, const hardkv_cache *cache,
+                  const void *k_new, const void *v_new, void *ws, cudaStream_t stream);
+
+/* Stage 4 (sec. 2.A Tier 3, "eviction or weighted merge"). For each sequence with
+ * moved[b] != 0, the block of positions [s_lo - block, s_lo) that just left the
+ * Sparse tier is, per KV head: EVICT — dropped (nothing to do); MERGE — folded token
+ * by token (position order) into the Condensed slot s >= n_sink with w_s > 0 of
+ * highest cosine similarity (ties -> lowest s): k_s <- (w_s k_s + k_x)/(w_s + 1),
+ * v_s likewise (float64 arithmetic, rounded to nearest even in the storage dtype),
+ * w_s += 1. Must follow the hardkv_append of the same step. */
+int hardkv_condense(const hardkv_desc *desc, const hardkv_cache *cache, void *ws,
+                    cudaStream_t stream);
+
+/* Stage 2 (sec. 2.B Logits Calibration; sec. 2.A Tier 2 calibrated top-p).
+ * For each selected (b,h) (select_mode), over the Sparse candidates j
+ * (positions s_lo + j < d_lo):
+ *   s_j = max_{g in group(h)} (q_g . k_j) / sqrt(d)       max-pooled logit
+ *   p_j = softmax_j(s_j / tau[b,h])                       calibration
+ *   keep the shortest prefix of the (s desc, position asc) order whose mass is
+ *   >= p (p = 1 keeps all), at most Cap of them.
+ * Writes mask[b,h,:] (device uint32 [B,H,mask_words]; bit j set = kept; bits past
+ * the Sparse length are 0). tau: device float [B,H] or NULL (all 1). */
+int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cache,
+                                const void *q, const float *tau, float p,
+                                int32_t select_mode, uint32_t *mask, void *ws,
+                                cudaStream_t stream);
+
+/* Stage 3 (sec. 2.C Index Regularization: Rewrite Cache + Flatten Index to the max
+ * length). For each selected (b,h): the kept candidates of `mask` (device, layout as
+ * above), in ascending position order, go to compact slots 0..n-1 — K and V rows
+ * copied from the ring, sp_idx[slot] = position — with n = min(popcount, Cap) (a
+ * larger mask keeps its first Cap, counted as a clamp); sp_idx[n..Cap) = -1;
+ * n_kept = n. Payload rows of pad slots are not written. */
+int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache,
+                      const uint32_t *mask, int32_t select_mode, void *ws,
+                      cudaStream_t stream);
+
+/* Decode attention over the three tiers (implied by sec. 1 / sec. 5: attention runs
+ * on the regularized layout). For each query head g of KV head h:
+ *   out = sum_t softmax_t(l_t) v_t over
+ *         Dense positions [d_lo, len)                    l = q.k / sqrt(d)
+ *       U compact slots < n_kept with sp_idx >= s_lo     l = q.k / sqrt(d)
+ *       U Condensed slots with w > 0                     l = q.k / sqrt(d) + ln w
+ * as one joint softmax (split-K partials combined by log-sum-exp).
+ * out: device float [B,Hq,d]. */
+int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache,
+                       const void *q, float *out, void *ws, cudaStream_t stream);
+
+/* One fused decode step (sec. 2.A four-stage pipeline): append, condense (MERGE
+ * only), score + calibration + top-p, then regularize fused with attention: the
+ * kept rows are gathered once, written to the compact layout and attended in the
+ * same pass. Results equal hardkv_append; hardkv_condense;
+ * hardkv_score_calibrate_topp; hardkv_regularize; hardkv_decode_attn.
+ * All pointers in `args` are device pointers. */
+int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
+                       const hardkv_step_args *args, void *ws, cudaStream_t stream);
+
+/* hardkv_decode_step with the per-step tensors in HOST memory (pinned memory makes
+ * the copies asynchronous): args->q, k_new, v_new and tau (if not NULL) are read from
+ * the host, args->out is written to the host; the copies and the step are enqueued
+ * on `stream` and the caller synchronises before reading `out`. args->mask, if not
+ * NULL, is a device pointer. Staging buffers live in the workspace. */
+int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
+                            const hardkv_step_args *host_args, void *ws,
+                            cudaStream_t stream);
+
+/* Human-readable text of a return code (for HARDKV_ECUDA: the last CUDA error seen
+ * by this thread). The string is static or thread-local; do not free it. */
+const char *hardkv_strerror(int code);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HARDKV_H */

@@ -1,0 +1,112 @@
+"""Helpers of the GPU parity tests: run the CUDA path through the C ABI and the fp64
+oracle on the same seeded inputs, and compare them."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from attention_kv_head_b200 import binding as B
+from attention_kv_head_b200 import synth
+from attention_kv_head_b200.cache import DecodeCache
+from oracle import hardkv_oracle as O
+
+# bf16 attention tolerance: max-abs 1e-2 and rel-L2 2e-3 (fixed by the target bounds);
+# fp32 inputs: the same arithmetic with fp32 storage -> 1e-4 / 1e-5.
+TOL = {"bf16": (1e-2, 2e-3), "f32": (1e-4, 1e-5)}
+
+
+def oracle_params(w: synth.Workload) -> O.Params:
+    return O.Params(w.head_dim, w.group, w.dense_window, w.condensed_slots, w.block,
+                    w.sparse_cap, w.n_sink, w.dtype, w.condense_mode)
+
+
+def oracle_unit(w: synth.Workload, st: synth.InitialState, b: int, h: int, steps: int = 1):
+    L0 = int(st.len0[b])
+    _, ke, _, ve = synth.unit_kv(w, b, h, 0, L0)
+    C = w.condensed_slots
+    return O.Unit(oracle_params(w), ke, ve, ke[:C], ve[:C], np.ones(C), L0, int(st.d_lo0[b]),
+                  int(st.s_lo0[b]), L0 + steps + 1)
+
+
+def mask_bits(mask_words_row: np.ndarray, L: int) -> np.ndarray:
+    """Local indices j < L whose bit is set in one unit's mask words."""
+    words = mask_words_row.astype(np.uint32)
+    bits = ((words[:, None] >> np.arange(32, dtype=np.uint32)[None, :]) & 1).reshape(-1)
+    return np.nonzero(bits[:L])[0]
+
+
+def rel_l2(a: np.ndarray, b: np.ndarray) -> float:
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def upload_step(dc: DecodeCache, w: synth.Workload, st: synth.InitialState, t: int):
+    qraw, qex = synth.queries(w, t)
+    kr, ke, vr, ve = synth.step_kv(w, st.lens, t)
+    return (dc.to_dev(qraw), dc.to_dev(kr), dc.to_dev(vr)), (qex, ke, ve)
+
+
+def storage_exact(a: np.ndarray, dtype: str) -> np.ndarray:
+    if dtype == "bf16":
+        return synth.bf16_bits_to_f64(a)
+    return a.astype(np.float64)
+
+
+def device_rows(t: torch.Tensor) -> np.ndarray:
+    """Device tensor of the cache dtype -> exact float64 numpy."""
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+class StepCompare:
+    """Accumulates the comparison of one step over units."""
+
+    def __init__(self, dtype):
+        self.atol, self.rtol = TOL[dtype]
+        self.flipped_units = 0
+        self.flipped_tokens = 0
+        self.units = 0
+        self.worst_abs = 0.0
+        self.worst_rel = 0.0
+
+    def selection(self, sel: O.Selection, p: float, gpu_kept: np.ndarray):
+        ok, nd = O.allowed_flips(sel, p, gpu_kept)
+        assert ok, f"mask differs beyond the flip rule ({nd} tokens)"
+        if nd:
+            self.flipped_units += 1
+            self.flipped_tokens += nd
+        return nd == 0
+
+    def attention(self, gpu: np.ndarray, ref: np.ndarray):
+        self.units += 1
+        a = float(np.abs(gpu - ref).max())
+        r = rel_l2(gpu, ref)
+        self.worst_abs = max(self.worst_abs, a)
+        self.worst_rel = max(self.worst_rel, r)
+        assert a <= self.atol and r <= self.rtol, (a, r)
+
+
+def run_unfused_step(dc: DecodeCache, q, k, v, p, select_mode=B.SELECT_ALL, tau=None):
+    dc.append(k, v)
+    dc.condense()
+    mask = dc.new_mask()
+    dc.score_calibrate_topp(q, p, mask, tau=tau, select_mode=select_mode)
+    dc.regularize(mask, select_mode=select_mode)
+    d = dc.desc
+    out = torch.empty(d.batch, d.n_q_heads, d.head_dim, dtype=torch.float32, device=dc.device)
+    dc.decode_attn(q, out)
+    return mask, out
+
+
+def run_fused_step(dc: DecodeCache, q, k, v, p, select_mode=B.SELECT_ALL, tau=None):
+    mask = dc.new_mask()
+    d = dc.desc
+    out = torch.empty(d.batch, d.n_q_heads, d.head_dim, dtype=torch.float32, device=dc.device)
+    dc.step(q, k, v, out, p, tau=tau, mask=mask, select_mode=select_mode)
+    return mask, out
+
+
+def scores_from_ws(dc: DecodeCache) -> np.ndarray:
+    """The workspace starts with the fp32 score array [B*H, R] (white-box check)."""
+    d = dc.desc
+    n = d.batch * d.n_kv_heads * d.ring_rows
+    return dc.ws[: n * 4].view(torch.float32).cpu().numpy().reshape(d.batch * d.n_kv_heads,
+                                                                     d.ring_rows)

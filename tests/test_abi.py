@@ -1,0 +1,113 @@
+"""The C-ABI library loads and exports every symbol include/hardkv.h declares, and its
+host-side validation returns the documented codes without touching a GPU."""
+import ctypes
+import subprocess
+
+import pytest
+
+from attention_kv_head_b200 import binding as B
+from attention_kv_head_b200 import build as Bd
+
+
+@pytest.fixture(scope="module")
+def lib():
+    Bd.build()
+    return B.load()
+
+
+def desc(**kw):
+    base = dict(batch=8, n_q_heads=32, n_kv_heads=8, head_dim=128, block=16, dense_window=200,
+                condensed_slots=256, n_sink=4, sparse_cap=7680, ring_rows=8000, dtype=B.BF16,
+                condense_mode=B.EVICT)
+    base.update(kw)
+    return B.Desc(**base)
+
+
+def test_every_declared_function_is_exported(lib):
+    names = B.header_functions()
+    assert len(names) >= 11
+    out = subprocess.run(["nm", "-D", "--defined-only", B.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for n in names:
+        assert n in exported, n
+        assert hasattr(lib, n)
+
+
+def test_north_star_entry_points_declared():
+    for n in ("hardkv_append", "hardkv_score_calibrate_topp", "hardkv_regularize",
+              "hardkv_condense", "hardkv_decode_attn"):
+        assert n in B.header_functions()
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dtype", 7, B.EDTYPE), ("batch", 0, B.EINVAL), ("n_q_heads", 12, B.EINVAL),
+    ("n_q_heads", 8 * 17, B.EINVAL), ("head_dim", 96, B.EINVAL), ("block", 0, B.EINVAL),
+    ("condensed_slots", 0, B.EINVAL), ("n_sink", 300, B.EINVAL), ("sparse_cap", 0, B.ECAP),
+    ("ring_rows", 8001, B.ECAP), ("ring_rows", 192, B.ECAP), ("dense_window", 1000, B.ECAP), ("condense_mode", 3, B.EINVAL),
+])
+def test_validate_rejects(lib, field, value, code):
+    d = desc(**{field: value})
+    assert lib.hardkv_validate(ctypes.byref(d)) == code
+    assert lib.hardkv_workspace_bytes(ctypes.byref(d)) == 0
+
+
+def test_validate_accepts_all_workloads(lib):
+    from attention_kv_head_b200 import synth
+    for w in synth.WORKLOADS.values():
+        d = B.Desc(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.block, w.dense_window,
+                   w.condensed_slots, w.n_sink, w.sparse_cap, w.derived_ring_rows(),
+                   B.BF16 if w.dtype == "bf16" else B.F32, w.condense_mode)
+        assert lib.hardkv_validate(ctypes.byref(d)) == B.OK, w.name
+        ws = lib.hardkv_workspace_bytes(ctypes.byref(d))
+        assert 0 < ws < 2 ** 31
+        assert lib.hardkv_mask_words(ctypes.byref(d)) * 32 >= d.ring_rows
+
+
+def test_merge_slot_limit(lib):
+    assert lib.hardkv_validate(ctypes.byref(desc(condense_mode=B.MERGE, condensed_slots=2048))) == B.OK
+    assert lib.hardkv_validate(ctypes.byref(desc(condense_mode=B.MERGE, condensed_slots=4096))) == B.EINVAL
+
+
+def _fake_cache(misalign=None, null=None):
+    vals = {}
+    for i, (name, _) in enumerate(B.Cache._fields_):
+        vals[name] = 0x10000 * (i + 1)
+    if misalign:
+        vals[misalign] += 4
+    if null:
+        vals[null] = None
+    return B.Cache(**vals)
+
+
+def test_entry_points_validate_before_any_launch(lib):
+    """Bad arguments return their code with nothing enqueued (fake pointers are never
+    dereferenced because validation fails first)."""
+    d = desc()
+    c = _fake_cache()
+    ws = ctypes.c_void_p(0x7000000)
+    assert lib.hardkv_append(ctypes.byref(d), None, 0x100, 0x200, ws, None) == B.EINVAL
+    assert lib.hardkv_append(ctypes.byref(d), ctypes.byref(_fake_cache(null="len")), 0x100, 0x200,
+                             ws, None) == B.EINVAL
+    assert lib.hardkv_append(ctypes.byref(d), ctypes.byref(_fake_cache(misalign="k_sp")), 0x100,
+                             0x200, ws, None) == B.EALIGN
+    assert lib.hardkv_append(ctypes.byref(d), ctypes.byref(c), 0x104, 0x200, ws, None) == B.EALIGN
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert lib.hardkv_score_calibrate_topp(ctypes.byref(d), ctypes.byref(c), 0x100, None,
+                                               ctypes.c_float(p), 0, 0x300, ws, None) == B.EINVAL
+    assert lib.hardkv_score_calibrate_topp(ctypes.byref(d), ctypes.byref(c), 0x100, None,
+                                           ctypes.c_float(0.9), 5, 0x300, ws, None) == B.EINVAL
+    assert lib.hardkv_regularize(ctypes.byref(d), ctypes.byref(c), None, 0, ws, None) == B.EINVAL
+    assert lib.hardkv_decode_attn(ctypes.byref(d), ctypes.byref(c), 0x100, None, ws, None) == B.EINVAL
+    bad = desc(dtype=9)
+    assert lib.hardkv_condense(ctypes.byref(bad), ctypes.byref(c), ws, None) == B.EDTYPE
+    assert lib.hardkv_decode_step(ctypes.byref(d), ctypes.byref(c), None, ws, None) == B.EINVAL
+    args = B.StepArgs(0x100, 0x200, 0x300, None, ctypes.c_float(2.0), 0, None, 0x400, None)
+    assert lib.hardkv_decode_step(ctypes.byref(d), ctypes.byref(c), ctypes.byref(args), ws,
+                                  None) == B.EINVAL
+    assert lib.hardkv_decode_step_host(ctypes.byref(d), ctypes.byref(c), None, ws, None) == B.EINVAL
+
+
+def test_strerror(lib):
+    for code in (B.OK, B.EINVAL, B.EALIGN, B.EDTYPE, B.ECAP, B.ECUDA, 12345):
+        assert isinstance(B.strerror(code), str) and B.strerror(code)

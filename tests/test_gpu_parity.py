@@ -1,0 +1,319 @@
+"""GPU (sm_100a) vs fp64 oracle on the same seeded inputs, through the C ABI.
+
+Bars: compaction indices, kept counts and boundaries bit-exact; masks identical except
+near-threshold tokens (oracle.allowed_flips, counted); attention max-abs <= 1e-2 and
+rel-L2 <= 2e-3 for bf16 (1e-4 / 1e-5 for fp32 storage); scores within 1e-5 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+from attention_kv_head_b200 import binding as B
+from attention_kv_head_b200 import synth
+from attention_kv_head_b200.cache import DecodeCache
+from oracle import hardkv_oracle as O
+from tests import gpu_util as U
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def oracle_unit_from_state(st: synth.InitialState, b: int, h: int, steps: int = 1):
+    """Oracle unit built from the very host arrays uploaded to the GPU."""
+    w = st.w
+    C, R = w.condensed_slots, st.R
+    L0 = int(st.len0[b])
+    K = np.zeros((L0, w.head_dim))
+    V = np.zeros((L0, w.head_dim))
+    K[:C] = U.storage_exact(st.k_cd[b, h], w.dtype)
+    V[:C] = U.storage_exact(st.v_cd[b, h], w.dtype)
+    pos = np.arange(C, L0)
+    K[C:] = U.storage_exact(st.k_ring[b, h, pos % R], w.dtype)
+    V[C:] = U.storage_exact(st.v_ring[b, h, pos % R], w.dtype)
+    return O.Unit(U.oracle_params(w), K, V, K[:C], V[:C], st.w_cd[b, h].astype(np.float64), L0,
+                  int(st.d_lo0[b]), int(st.s_lo0[b]), L0 + steps + 1)
+
+
+SMALL = {
+    "bf16_d128_g4": synth.small(),
+    "bf16_d64_g5": synth.small(n_q_heads=10, n_kv_heads=2, head_dim=64),
+    "f32_d64_g1": synth.small(dtype=synth.F32, n_q_heads=2, n_kv_heads=2, head_dim=64),
+    "f32_d128_g4": synth.small(dtype=synth.F32),
+    "bf16_g16": synth.small(n_q_heads=32, n_kv_heads=2),
+    "bf16_g8_d64": synth.small(n_q_heads=16, n_kv_heads=2, head_dim=64, temp_range=(2.0, 6.0)),
+    "clamp": synth.small(sparse_cap=100),
+    "keep_all": synth.small(p=1.0),
+    "keep_all_clamped": synth.small(p=1.0, sparse_cap=50),
+    "ring_wrap": synth.small(context=1000, condensed_slots=400),
+    "no_sparse": synth.small(context=72, dense_window=48, condensed_slots=24),
+    "p_low": synth.small(p=0.3, temp_range=(0.25, 8.0)),
+    "batch5": synth.small(batch=5, context=333, sparse_cap=250),
+}
+
+
+def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_expected=None):
+    G = w.group
+    m = mask.cpu().numpy().view(np.uint32)
+    n_kept = dc.n_kept.cpu().numpy()
+    sp_idx = dc.sp_idx.cpu().numpy()
+    k_sp = U.device_rows(dc.k_sp)
+    v_sp = U.device_rows(dc.v_sp)
+    o = out.cpu().numpy()
+    lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
+    for (b, h), unit in units.items():
+        res = unit.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, p)
+        assert (lens[b], dlo[b], slo[b]) == (unit.len, unit.d_lo, unit.s_lo)
+        L = unit.d_lo - unit.s_lo
+        kept = U.mask_bits(m[b, h], L)
+        allbits = U.mask_bits(m[b, h], m.shape[-1] * 32)
+        assert np.all(allbits < L)                      # no bit past the Sparse length
+        n = int(n_kept[b, h])
+        assert n == min(kept.size, w.sparse_cap) == kept.size
+        assert np.array_equal(sp_idx[b, h, :n], unit.s_lo + kept)
+        assert np.all(sp_idx[b, h, n:] == -1)
+        # compact rows are byte-identical to the raw rows of those positions
+        assert np.array_equal(k_sp[b, h, :n], unit.K[sp_idx[b, h, :n]])
+        assert np.array_equal(v_sp[b, h, :n], unit.V[sp_idx[b, h, :n]])
+        same = cmp.selection(res.sel, p, kept) if res.sel is not None else True
+        if same:
+            assert n == res.n and np.array_equal(sp_idx[b, h], res.idx)
+            cmp.attention(o[b, h * G:(h + 1) * G], res.out)
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_step_unfused_vs_oracle_and_fused(name):
+    w = SMALL[name]
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    dc2 = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    p = synth.p_values(w)[0]
+    mask, out = U.run_unfused_step(dc, q, k, v, p)
+    mask2, out2 = U.run_fused_step(dc2, q, k, v, p)
+    torch.cuda.synchronize()
+    units = {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
+             for h in range(w.n_kv_heads)}
+    # scores (white box): fp32 vs fp64 within 1e-5 relative to the unit's scale
+    sc = U.scores_from_ws(dc)
+    for (b, h), un in units.items():
+        L = int(st.d_lo0[b] - st.s_lo0[b])
+        if L == 0:
+            continue
+        ref = O.score(q_ex[b, h * w.group:(h + 1) * w.group], un.K[un.s_lo:un.d_lo])
+        got = sc[b * w.n_kv_heads + h, :L]
+        assert np.allclose(got, ref, rtol=1e-5, atol=1e-5 * np.abs(ref).max()), name
+    cmp = U.StepCompare(w.dtype)
+    compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp)
+    # fused step == unfused path, bit for bit
+    assert torch.equal(mask, mask2)
+    assert torch.equal(dc.n_kept, dc2.n_kept) and torch.equal(dc.sp_idx, dc2.sp_idx)
+    for t1, t2 in ((dc.len, dc2.len), (dc.d_lo, dc2.d_lo), (dc.s_lo, dc2.s_lo)):
+        assert torch.equal(t1, t2)
+    n = dc.n_kept.cpu().numpy()
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            assert torch.equal(dc.k_sp[b, h, :n[b, h]], dc2.k_sp[b, h, :n[b, h]])
+            assert torch.equal(dc.v_sp[b, h, :n[b, h]], dc2.v_sp[b, h, :n[b, h]])
+    assert torch.equal(out, out2)
+    st_words = dc.read_status()
+    assert st_words[B.ST_FLAGS] == 0
+    assert st_words[B.ST_SELECTIONS] == w.units
+    print(name, "flipped units", cmp.flipped_units, "worst abs", cmp.worst_abs, "rel", cmp.worst_rel)
+
+
+@pytest.mark.parametrize("frac,cap", [(0.3, 600), (0.9, 200), (0.0, 600), (1.0, 600)])
+@pytest.mark.parametrize("dtype", [synth.BF16, synth.F32])
+def test_regularize_and_attention_given_mask(frac, cap, dtype):
+    """A seeded mask drives both sides: compaction bit-exact, attention within tolerance."""
+    w = synth.small(dtype=dtype, sparse_cap=cap)
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    dc.append(k, v)
+    masks = {}
+    mask_np = np.zeros((w.batch, w.n_kv_heads, dc.mask_words), np.uint32)
+    for b in range(w.batch):
+        L = int(st.d_lo0[b] - st.s_lo0[b])
+        for h in range(w.n_kv_heads):
+            mk = synth.random_mask(w, b, h, L, frac)
+            masks[b, h] = mk
+            bits = np.zeros(dc.mask_words * 32, np.uint32)
+            bits[:L] = mk
+            mask_np[b, h] = (bits.reshape(-1, 32) << np.arange(32, dtype=np.uint32)).sum(1)
+            # bits past the Sparse length must be ignored by the kernel
+            mask_np[b, h, -1] |= np.uint32(0x80000000)
+    mask = torch.from_numpy(mask_np.view(np.int32)).to(dc.device)
+    dc.regularize(mask)
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, device=dc.device)
+    dc.decode_attn(q, out)
+    torch.cuda.synchronize()
+    n_kept = dc.n_kept.cpu().numpy()
+    sp_idx = dc.sp_idx.cpu().numpy()
+    k_sp, v_sp = U.device_rows(dc.k_sp), U.device_rows(dc.v_sp)
+    o = out.cpu().numpy()
+    cmp = U.StepCompare(dtype)
+    clamps = 0
+    for b in range(w.batch):
+        for h in range(w.n_kv_heads):
+            un = oracle_unit_from_state(st, b, h)
+            un.append(k_ex[b, h], v_ex[b, h])
+            pos = np.arange(un.s_lo, un.d_lo)
+            n, idx, kc, vc = O.regularize(masks[b, h], pos, un.K[un.s_lo:un.d_lo],
+                                          un.V[un.s_lo:un.d_lo], cap)
+            clamps += int(masks[b, h].sum() > cap)
+            assert n_kept[b, h] == n
+            assert np.array_equal(sp_idx[b, h], idx)
+            assert np.array_equal(k_sp[b, h, :n], kc) and np.array_equal(v_sp[b, h, :n], vc)
+            un.n, un.idx, un.sp_k, un.sp_v = n, idx, kc, vc
+            cmp.attention(o[b, h * w.group:(h + 1) * w.group],
+                          un.attend(q_ex[b, h * w.group:(h + 1) * w.group]))
+    assert dc.read_status()[B.ST_CLAMPS] == clamps
+
+
+def test_uniform_and_one_hot_heads():
+    """Planted keys: a head whose candidates are all equal keeps ceil(p n) lowest
+    positions; a head with one dominant key keeps exactly that key."""
+    w = synth.small(batch=1, n_kv_heads=2, n_q_heads=8, p=0.6)
+    st = synth.initial_state(w)
+    R, C = st.R, w.condensed_slots
+    L0 = int(st.len0[0])
+    pos = np.arange(C, L0)
+    st.k_ring[0, 0, pos % R] = st.k_ring[0, 0, C % R]        # head 0: all keys identical
+    hot = int(C + (L0 - C) // 3)
+    st.k_ring[0, 1, pos % R] = 0                              # head 1: zero keys ...
+    st.k_ring[0, 1, hot % R] = synth.to_bf16_bits(np.full(w.head_dim, 30.0, np.float32))
+    dc = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    qh = q_ex.copy()
+    # make every query of head 1 positive so the planted key dominates
+    q_dev = q.clone()
+    q_dev[0, 4:8] = q_dev[0, 4:8].abs()
+    qh[0, 4:8] = np.abs(qh[0, 4:8])
+    mask, out = U.run_unfused_step(dc, q_dev, k, v, w.p)
+    torch.cuda.synchronize()
+    m = mask.cpu().numpy().view(np.uint32)
+    L = int(dc.d_lo[0] - dc.s_lo[0])
+    kept0 = U.mask_bits(m[0, 0], L)
+    p32 = float(np.float32(w.p))
+    assert kept0.tolist() == list(range(int(np.ceil(p32 * L))))
+    kept1 = U.mask_bits(m[0, 1], L)
+    assert kept1.tolist() == [hot - C]
+    for h in range(2):
+        un = oracle_unit_from_state(st, 0, h)
+        res = un.step(qh[0, h * 4:(h + 1) * 4], k_ex[0, h], v_ex[0, h], 1.0, w.p)
+        assert res.sel.kept.tolist() == (kept0 if h == 0 else kept1).tolist()
+
+
+@pytest.mark.parametrize("mode", [synth.MERGE, synth.EVICT])
+@pytest.mark.parametrize("select", ["all", "moved"])
+def test_multistep_small(mode, select):
+    """40 steps: block moves every 16 steps, merges into the Condensed tier, per-step
+    parity of boundaries, masks, compaction, Condensed state and attention."""
+    w = synth.small(condense_mode=mode, steps=40, batch=2, context=300 + 0)
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    units = {(b, h): oracle_unit_from_state(st, b, h, steps=w.steps) for b in range(w.batch)
+             for h in range(w.n_kv_heads)}
+    sel_mode = B.SELECT_ALL if select == "all" else B.SELECT_MOVED
+    cmp = U.StepCompare(w.dtype)
+    G = w.group
+    diverged = set()
+    for t in range(w.steps):
+        (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, t)
+        if t == 0 and select == "moved":
+            mask, out = U.run_fused_step(dc, q, k, v, w.p, select_mode=B.SELECT_ALL)
+            rs = "all"
+        else:
+            mask, out = U.run_fused_step(dc, q, k, v, w.p, select_mode=sel_mode)
+            rs = select
+        torch.cuda.synchronize()
+        m = mask.cpu().numpy().view(np.uint32)
+        n_kept, sp_idx = dc.n_kept.cpu().numpy(), dc.sp_idx.cpu().numpy()
+        k_cd, v_cd = U.device_rows(dc.k_cd), U.device_rows(dc.v_cd)
+        w_cd = dc.w_cd.cpu().numpy()
+        o = out.cpu().numpy()
+        bounds = [t_.cpu().numpy() for t_ in (dc.len, dc.d_lo, dc.s_lo, dc.moved)]
+        for (b, h), un in units.items():
+            if (b, h) in diverged:
+                continue
+            res = un.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, w.p, reselect=rs)
+            assert (bounds[0][b], bounds[1][b], bounds[2][b], bool(bounds[3][b])) == \
+                (un.len, un.d_lo, un.s_lo, res.moved)
+            if res.merge is not None and res.merge.gaps and min(res.merge.gaps) <= 1e-6:
+                diverged.add((b, h))      # a near-tie may legitimately pick another slot
+                continue
+            assert np.array_equal(w_cd[b, h], un.cd_w.astype(np.float32))
+            assert np.array_equal(k_cd[b, h], un.cd_k) and np.array_equal(v_cd[b, h], un.cd_v)
+            same = True
+            if res.sel is not None:
+                L = un.d_lo - un.s_lo
+                same = cmp.selection(res.sel, w.p, U.mask_bits(m[b, h], L))
+            if same:
+                assert n_kept[b, h] == un.n and np.array_equal(sp_idx[b, h], un.idx)
+                cmp.attention(o[b, h * G:(h + 1) * G], res.out)
+    assert dc.read_status()[B.ST_FLAGS] == 0
+    assert len(diverged) <= 1
+
+
+@pytest.mark.parametrize("name", ["pr1", "llama8b_8k"])
+def test_full_size_single_step(name):
+    """The single-step workloads at full size, every unit against the oracle."""
+    w = synth.WORKLOADS[name]
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    mask, out = U.run_fused_step(dc, q, k, v, w.p)
+    torch.cuda.synchronize()
+    units = {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
+             for h in range(w.n_kv_heads)}
+    cmp = U.StepCompare(w.dtype)
+    compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, w.p, cmp)
+    assert cmp.flipped_units <= max(1, w.units // 50)
+    print(name, "flipped", cmp.flipped_units, cmp.flipped_tokens, "abs", cmp.worst_abs,
+          "rel", cmp.worst_rel, "kept", dc.n_kept.sum().item())
+
+
+def test_graph_capture_replays_the_step():
+    w = synth.small(batch=3)
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    (q, k, v), _ = U.upload_step(dc, w, st, 0)
+    snap = dc.snapshot_bounds()
+    mask_e, out_e = U.run_fused_step(dc, q, k, v, w.p)
+    torch.cuda.synchronize()
+    mask_e, out_e = mask_e.clone(), out_e.clone()
+    dc.restore_bounds(snap)
+    mask = dc.new_mask()
+    out = torch.empty_like(out_e)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        dc.step(q, k, v, out, w.p, mask=mask, stream=s)   # warm-up (sets kernel attributes)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    dc.restore_bounds(snap)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        dc.step(q, k, v, out, w.p, mask=mask)
+    for _ in range(3):
+        dc.restore_bounds(snap)
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, out_e) and torch.equal(mask, mask_e)
+
+
+def test_host_entry_point_matches_device_step():
+    w = synth.small(batch=2)
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    dc2 = DecodeCache.from_state(st)
+    (q, k, v), _ = U.upload_step(dc, w, st, 0)
+    _, out = U.run_fused_step(dc, q, k, v, w.p)
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    dc2.step_host(qh, kh, vh, oh, w.p)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, out.cpu())
