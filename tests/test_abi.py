@@ -44,7 +44,7 @@ def test_north_star_entry_points_declared():
     ("dtype", 7, B.EDTYPE), ("batch", 0, B.EINVAL), ("n_q_heads", 12, B.EINVAL),
     ("n_q_heads", 8 * 17, B.EINVAL), ("head_dim", 96, B.EINVAL), ("block", 0, B.EINVAL),
     ("condensed_slots", 0, B.EINVAL), ("n_sink", 300, B.EINVAL), ("sparse_cap", 0, B.ECAP),
-    ("ring_rows", 8001, B.ECAP), ("ring_rows", 192, B.ECAP), ("dense_window", 1000, B.ECAP), ("condense_mode", 3, B.EINVAL),
+    ("ring_rows", 8001, B.ECAP), ("ring_rows", 192, B.ECAP), ("dense_window", 7990, B.ECAP), ("condense_mode", 3, B.EINVAL),
 ])
 def test_validate_rejects(lib, field, value, code):
     d = desc(**{field: value})
