@@ -1,0 +1,438 @@
+"""Benchmark of the HARD-KV decode step (one attention layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path (append, condense on block steps, score +
+calibration + top-p, regularize fused with attention, combine) over one batch of
+synthetic input, replayed from the same starting cache state so every timed step is
+the workload's single decode step. Each step is one CUDA-graph replay timed with CUDA
+events on the launching stream; L2 is flushed (a 2 x L2 write) before every timed
+step, outside the timed events. `e2e` repeats the measurement through the host-buffer
+C entry point (hardkv_decode_step_host: pinned H2D of q / k_new / v_new, the step,
+D2H of the output). With --gpus N (torchrun) every rank runs an independent replica of
+the workload on its own GPU (no collective in the step) and the step time is the max
+over ranks.
+
+`--impl reference` times the fp64 CPU oracle as it stands, on this host's cores, on a
+bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "compressed-KV decode tokens/s at batch×ctx; HBM GB/s as % of B200 peak"
+L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0
+STAGES = ("append", "condense", "score", "topp", "attend", "combine")
+KERNEL_OF_STAGE = {"append": "append_kernel", "condense": "condense_kernel",
+                   "score": "score_tma_kernel", "topp": "topp_kernel",
+                   "attend": "attend_kernel", "combine": "combine_kernel"}
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "attention_kv_head_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu capture of the current sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+        e = d.get(kernel)
+        if e and e.get("csrc_sha") == csrc_digest() and e.get("workload") == workload:
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+    return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons (NVML) while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.index, self.period, self.samples = index, period_s, []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+                rs = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        busy = [m for m, r in self.samples if not (r & 0x1)] or [m for m, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples)}
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_max(x: float, world: int, device=None) -> float:
+    """Max of a float over ranks (identity when not distributed)."""
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- bytes
+
+def algorithmic_bytes(w, n_kept: np.ndarray, lens, d_lo, s_lo) -> dict:
+    """Bytes each stage must move (reads + writes), from the device-side kept counts."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, H, G, C = w.head_dim, w.n_kv_heads, w.group, w.condensed_slots
+    Ls = (d_lo - s_lo).astype(np.int64)                      # per sequence
+    dense = (lens - d_lo).astype(np.int64)
+    U = w.batch * H
+    sum_Ls = int(Ls.sum()) * H
+    sum_n = int(n_kept.sum())
+    sum_dense = int(dense.sum()) * H
+    q = w.batch * w.n_q_heads * d * e
+    by = {
+        "append": 2 * U * d * e * 2,                                   # read k_new,v_new; write rows
+        "condense": 0,
+        "score": sum_Ls * d * e + q + sum_Ls * 4,                      # keys + q + scores
+        "topp": sum_Ls * 4 + sum_Ls // 8 + sum_n * 4,                  # scores + mask + idx
+        "attend": sum_n * 2 * d * e * 2 + sum_n * 4                    # gather read + compact write
+                  + (sum_dense + U * C) * 2 * d * e + U * C * 4 + q,  # Dense + Condensed
+        "combine": w.batch * w.n_q_heads * d * 4,
+    }
+    by["total"] = sum(by.values())
+    by["sum_kept"] = sum_n
+    by["kept_fraction"] = sum_n / max(sum_Ls, 1)
+    return by
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, world, rank, local) -> dict:
+    import torch
+
+    from attention_kv_head_b200 import binding as Bn
+    from attention_kv_head_b200 import build as Bd
+    from attention_kv_head_b200 import synth
+    from attention_kv_head_b200.cache import DecodeCache
+
+    Bd.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = synth.WORKLOADS[args.workload].with_(seed=rank)
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st, device=dev)
+    qraw, _ = synth.queries(w, 0)
+    kr, _, vr, _ = synth.step_kv(w, st.lens, 0)
+    q, k, v = dc.to_dev(qraw), dc.to_dev(kr), dc.to_dev(vr)
+    p = synth.p_values(w)[0]
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dev)
+    mask = dc.new_mask()
+    snap = dc.snapshot_bounds()
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(Bn.STEP_EVENTS)]
+    with torch.cuda.stream(stream):
+        for e_ in evs:
+            e_.record(stream)                      # create the CUDA events
+        for _ in range(2):                         # eager warm-up (sets kernel attributes)
+            dc.restore_bounds(snap)
+            dc.step(q, k, v, out, p, mask=mask, events=evs, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    dc.restore_bounds(snap)
+    with torch.cuda.graph(g, stream=stream):
+        dc.step(q, k, v, out, p, mask=mask, events=evs)
+    kernels_per_step = 5 + (1 if w.condense_mode == synth.MERGE else 0)
+
+    def one_step(timed: bool):
+        with torch.cuda.stream(stream):
+            dc.restore_bounds(snap)
+            flush.zero_()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            g.replay()
+            t1.record(stream)
+        stream.synchronize()
+        if not timed:
+            return None
+        st_ms = [evs[i].elapsed_time(evs[i + 1]) for i in range(len(STAGES))]
+        return t0.elapsed_time(t1), st_ms
+
+    for _ in range(args.warmup):
+        one_step(False)
+    step_ms, stage_ms = [], []
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for _ in range(args.steps):
+            a, b = one_step(True)
+            step_ms.append(a)
+            stage_ms.append(b)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    mean_ms = float(np.mean(step_ms))
+    max_ms = dist_max(mean_ms, world, dev)
+
+    # kept counts of this step (device) -> algorithmic bytes
+    lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
+    by = algorithmic_bytes(w, dc.n_kept.cpu().numpy(), lens, dlo, slo)
+    stage_mean = {s: float(np.mean([x[i] for x in stage_ms])) for i, s in enumerate(STAGES)}
+
+    # e2e through the host-buffer entry point
+    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    e2e_ms = []
+    for i in range(args.warmup + args.steps):
+        with torch.cuda.stream(stream):
+            dc.restore_bounds(snap)
+            flush.zero_()
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            dc.step_host(qh, kh, vh, oh, p, mask=mask, stream=stream)
+            t1.record(stream)
+        stream.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(t0.elapsed_time(t1))
+    e2e_mean = dist_max(float(np.mean(e2e_ms)), world, dev)
+    status = dc.read_status()
+    del g
+    return dict(w=w, mean_ms=mean_ms, max_ms=max_ms, bytes=by, stages=stage_mean,
+                clocks=clk.summary(), e2e_ms=e2e_mean, kernels_per_step=kernels_per_step,
+                h2d=int(q.numel() * q.element_size() + 2 * k.numel() * k.element_size()),
+                d2h=int(out.numel() * 4), status=status, p50_ms=float(np.median(step_ms)))
+
+
+# ----------------------------------------------------------------------------- oracle
+
+_ORACLE_CACHE: dict = {}
+
+
+def oracle_inputs(w):
+    """Per-unit exact inputs of the workload's first decode step (generated once)."""
+    if w.name in _ORACLE_CACHE:
+        return _ORACLE_CACHE[w.name]
+    from attention_kv_head_b200 import synth
+    lens = synth.seq_lengths(w)
+    _, q_ex = synth.queries(w, 0)
+    _, k_ex, _, v_ex = synth.step_kv(w, lens, 0)
+    G = w.group
+    units = []
+    for b in range(w.batch):
+        L0 = int(lens[b]) - 1
+        for h in range(w.n_kv_heads):
+            _, ke, _, ve = synth.unit_kv(w, b, h, 0, L0)
+            units.append((b, h, L0, ke, ve, q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h]))
+    _ORACLE_CACHE[w.name] = units
+    return units
+
+
+def oracle_timing(w, budget_s: float) -> dict:
+    """Time the oracle's decode step on whole steps (all (sequence, KV-head) units of the
+    workload's first step) repeated until `budget_s` of oracle time; at least one unit."""
+    from attention_kv_head_b200 import synth
+    from oracle import hardkv_oracle as O
+    p = synth.p_values(w)[0]
+    prm = O.Params(w.head_dim, w.group, w.dense_window, w.condensed_slots, w.block,
+                   w.sparse_cap, w.n_sink, w.dtype, w.condense_mode)
+    C = w.condensed_slots
+    units = oracle_inputs(w)
+    done, elapsed = 0, 0.0
+    while elapsed < budget_s:
+        for (b, h, L0, ke, ve, qg, kx, vx) in units:
+            un = O.Unit(prm, ke, ve, ke[:C], ve[:C], np.ones(C), L0, L0 + 1 - w.dense_window,
+                        C, L0 + 2)
+            t = time.perf_counter()
+            un.step(qg, kx, vx, 1.0, p)
+            elapsed += time.perf_counter() - t
+            done += 1
+            if elapsed >= budget_s:
+                break
+    step_s = elapsed / done * len(units)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = 1
+    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": int(cores),
+            "kind": "oracle", "seconds": round(elapsed, 3),
+            "sample": f"{done} (sequence, KV-head) unit steps of the {w.name} decode step "
+                      f"({len(units)} units per step); step time = mean unit time x {len(units)}"}
+
+
+# ----------------------------------------------------------------------------- main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="llama8b_8k")
+    ap.add_argument("--impl", default="hardkv", choices=["hardkv", "reference"])
+    ap.add_argument("--oracle-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_info()
+    from attention_kv_head_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    config = {"workload": w.name, "batch": w.batch, "context": w.context,
+              "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
+              "dense_window": w.dense_window, "condensed_slots": w.condensed_slots,
+              "sparse_cap": w.sparse_cap, "p": synth.p_values(w)[0],
+              "l2": "flushed (2 x L2 write) before every timed step",
+              "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        per_step = max(0.2, min(10.0, 60.0 / max(args.steps + args.warmup, 1)))
+        vals, cb = [], None
+        for i in range(args.warmup + args.steps):
+            cb = oracle_timing(w, per_step)
+            if i >= args.warmup:
+                vals.append(cb["value"])
+        v = float(np.mean(vals))
+        cb["value"] = v
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": 1e3 * w.batch / v, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    r = run_gpu(args, world, rank, local)
+    peaks = measured_peaks()
+    by = r["bytes"]
+    # dominant kernel by time
+    dom = max(("score", "topp", "attend"), key=lambda s: r["stages"][s])
+    dom_us = r["stages"][dom] * 1e3
+    achieved = by[dom] / (dom_us * 1e-6) / 1e9
+    traffic = ncu_traffic(KERNEL_OF_STAGE[dom], w.name)
+    step_gbs = by["total"] / (r["mean_ms"] * 1e-3) / 1e9
+    value = world * w.batch / (r["max_ms"] * 1e-3)
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["max_ms"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16"
+        if w.dtype == "bf16" else "f32", "data": "synthetic", "config": config,
+        "e2e": {"value": world * w.batch / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "ms_per_step": r["e2e_ms"], "api": "hardkv_decode_step_host"},
+        "roofline": {"bound": "hbm", "kernel": KERNEL_OF_STAGE[dom], "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "alg_bytes_per_launch": by[dom],
+                     "launch_us": dom_us, "peak_source": peaks["source"]},
+        "step_hbm": {"alg_bytes": by["total"], "gbs": step_gbs,
+                     "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
+                     "frac_of_measured": step_gbs / peaks["hbm_gbs"],
+                     "kept_fraction": by["kept_fraction"], "sum_kept": by["sum_kept"],
+                     "p50_ms": r["p50_ms"]},
+        "stages_us": {s: round(v_ * 1e3, 2) for s, v_ in r["stages"].items()},
+        "stage_alg_bytes": {s: by[s] for s in STAGES},
+        "gpu_launches": r["kernels_per_step"] * args.steps,
+        "clocks": r["clocks"],
+        "device_status": [int(x) for x in r["status"]],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = oracle_timing(w, args.oracle_seconds)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
