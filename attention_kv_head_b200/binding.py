@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libhardkv.so")
 HEADER = os.path.join(HERE, "..", "include", "hardkv.h")
 
-OK, EINVAL, EALIGN, EDTYPE, ECAP, ECUDA = 0, -1, -2, -3, -4, -5
+OK, EINVAL, EALIGN, EDTYPE, ECAP, ECUDA, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
 F32, BF16 = 0, 1
 EVICT, MERGE = 0, 1
 SELECT_ALL, SELECT_MOVED = 0, 1
@@ -70,6 +70,9 @@ _SIGS = {
     "hardkv_decode_step_host": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),
                                                ctypes.POINTER(StepArgs), _vp, _vp]),
     "hardkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "hardkv_score_calibrate_topp_static": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),
+                                                          _vp, _vp, ctypes.c_float, _i32, _vp, _vp]),
+    "hardkv_static_scratch_bytes": (ctypes.c_size_t, []),
 }
 
 

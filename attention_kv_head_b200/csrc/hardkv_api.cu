@@ -533,8 +533,76 @@ const char *hardkv_strerror(int code) {
     case HARDKV_EDTYPE: return "unsupported dtype";
     case HARDKV_ECAP: return "capacity rule broken (sparse_cap < 1, ring_rows too small or not a multiple of 64)";
     case HARDKV_ECUDA: return g_err;
+    case HARDKV_ESCRATCH: return g_err;
     default: return "unknown hardkv error code";
   }
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- allocation-free variant
+//
+// hardkv_score_calibrate_topp_static: the score / calibration / top-p stage for callers
+// that cannot allocate device memory. Its scratch (the fp32 score array and the
+// per-tile maxima) lives in this file-scope device array instead of a caller workspace.
+// The array is a device symbol: on the host its name is only a stand-in, so the host
+// asks the runtime for its device address (once per device) and passes that pointer.
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(32) << 20;  // 32 MiB per device
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+// Device address of g_static_scratch on the current device (looked up once per device).
+int static_scratch(void **out) {
+  static void *addr[64] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return HARDKV_EINVAL;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress");
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return HARDKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t hardkv_static_scratch_bytes(void) { return kStaticScratchBytes; }
+
+int hardkv_score_calibrate_topp_static(const hardkv_desc *desc, const hardkv_cache *cache,
+                                       const void *q, const float *tau, float p,
+                                       int32_t select_mode, uint32_t *mask, cudaStream_t stream) {
+  HKV_TRY(validate_desc(desc));
+  HKV_TRY(check_cache(cache));
+  HKV_TRY(check_ptr(q));
+  HKV_TRY(check_ptr(tau, true));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_p(p));
+  HKV_TRY(check_mode(select_mode));
+  const Layout L = layout(desc);
+  const size_t U = (size_t)desc->batch * desc->n_kv_heads;
+  const size_t need = L.tile_max + U * (size_t)L.tm_stride * 4;  // scores, then tile maxima
+  if (need > kStaticScratchBytes) {
+    snprintf(g_err, sizeof(g_err),
+             "problem needs %zu bytes of score scratch, the built-in scratch holds %zu", need,
+             kStaticScratchBytes);
+    return HARDKV_ESCRATCH;
+  }
+  void *ws = nullptr;
+  HKV_TRY(static_scratch(&ws));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(cache);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, stream));
+  return launch_topp<false>(sh, c, ws, L, tau, p, select_mode, mask, stream);
 }
 
 }  // extern "C"

@@ -53,6 +53,8 @@ extern "C" {
 #define HARDKV_EDTYPE (-3)   /* dtype not HARDKV_F32 / HARDKV_BF16 */
 #define HARDKV_ECAP   (-4)   /* capacity rule broken (Cap < 1, R too small, R % 64) */
 #define HARDKV_ECUDA  (-5)   /* a CUDA launch or copy failed */
+#define HARDKV_ESCRATCH (-6) /* too large for the built-in scratch of the allocation-free
+                                entry point (hardkv_score_calibrate_topp_static) */
 
 enum { HARDKV_F32 = 0, HARDKV_BF16 = 1 };
 enum { HARDKV_EVICT = 0, HARDKV_MERGE = 1 };
@@ -209,6 +211,37 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
                             const hardkv_step_args *host_args, void *ws,
                             cudaStream_t stream);
+
+/* Allocation-free variant of hardkv_score_calibrate_topp (no counterpart in the
+ * paper: it only changes where the stage's scratch lives).
+ *
+ * Some callers cannot call cudaMalloc or hand this library a workspace: a plugin
+ * inside a host framework whose caching allocator owns all device memory and offers
+ * no scratch to this stage, code that runs while another component holds a stream
+ * capture in a mode that forbids allocation, or a latency-critical loop that cannot
+ * afford the synchronisation an allocation may cause. For them this entry point
+ * takes the same inputs and outputs as hardkv_score_calibrate_topp (q, tau, p,
+ * select_mode, mask: device pointers, same layouts and results) but no workspace:
+ * the fp32 score array and the per-tile maxima live in a file-scope device array of
+ * hardkv_static_scratch_bytes() bytes (32 MiB) that every GPU which loads the library
+ * holds until the process exits. It calls no cudaMalloc, cudaFree or allocating
+ * library routine.
+ *  - Limit: B*H*ring_rows*4 bytes of scores plus the tile maxima must fit in that
+ *    array; larger problems return HARDKV_ESCRATCH (nothing is enqueued).
+ *  - The first call on a device looks up the array's device address with
+ *    cudaGetSymbolAddress while that device is current; make that first call before
+ *    any stream capture that includes this entry point.
+ *  - Every call, on every stream, shares the one array and leaves its contents there;
+ *    nothing in it needs to start at zero (each call writes what it reads). Calls whose
+ *    executions overlap on the GPU race on the array: serialise them (one stream, or
+ *    events). */
+int hardkv_score_calibrate_topp_static(const hardkv_desc *desc, const hardkv_cache *cache,
+                                       const void *q, const float *tau, float p,
+                                       int32_t select_mode, uint32_t *mask,
+                                       cudaStream_t stream);
+
+/* Size in bytes of the built-in scratch used by hardkv_score_calibrate_topp_static. */
+size_t hardkv_static_scratch_bytes(void);
 
 /* Human-readable text of a return code (for HARDKV_ECUDA: the last CUDA error seen
  * by this thread). The string is static or thread-local; do not free it. */
