@@ -21,7 +21,7 @@ SELECT_ALL, SELECT_MOVED = 0, 1
 STATUS_WORDS = 8
 ST_FLAGS, ST_CLAMPS, ST_NEAR_TIES, ST_MERGED, ST_MOVES, ST_SELECTIONS = range(6)
 DEV_RING_OVERFLOW, DEV_BAD_BOUNDS, DEV_SEGMENTS, DEV_WAIT_TIMEOUT = 1, 2, 4, 8
-STEP_EVENTS = 7
+STEP_EVENTS = 6
 
 _i32 = ctypes.c_int32
 _vp = ctypes.c_void_p

@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "k_attend.cuh"
+#include "k_attend_bulk.cuh"
 #include "k_score.cuh"
 #include "k_select.cuh"
 #include "k_state.cuh"
@@ -36,8 +37,9 @@ int cuda_fail(cudaError_t e, const char *what) {
     if (r_ != HARDKV_OK) return r_; \
   } while (0)
 
-constexpr int kMinAttendCtas = 444;  // 3 resident attend CTAs x 148 SMs on B200
+constexpr int kAttendWave = 296;  // 2 resident attend CTAs x 148 SMs on B200
 constexpr size_t kMaxSmem = 227 * 1024;
+constexpr int kToppCacheMax = 40960;  // fp32 scores cached per top-p CTA (160 KB)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -87,7 +89,7 @@ Shape make_shape(const hardkv_desc *d) {
 }
 
 struct Layout {
-  size_t scores, tile_max, part, pre, st_q, st_k, st_v, st_out, st_tau, total;
+  size_t scores, tile_max, part, counters, st_q, st_k, st_v, st_out, st_tau, total;
   int tm_stride, P;
 };
 
@@ -98,10 +100,11 @@ Layout layout(const hardkv_desc *d) {
   L.tm_stride = kPartsPerTile * (d->ring_rows / kTile + 2);
   const long long rows_max =
       (long long)U * (d->sparse_cap + d->dense_window + d->block + d->condensed_slots);
+  // every unit has >= W + C rows, so a CTA range of <= (kSegMax - 1) (W + C) rows meets
+  // at most kSegMax units; P is that bound rounded up to whole waves
   const long long minrows = d->dense_window + d->condensed_slots;
-  long long P = (rows_max + 3 * minrows - 1) / (3 * minrows);
-  if (P < kMinAttendCtas) P = kMinAttendCtas;
-  L.P = (int)P;
+  const long long pmin = (rows_max + (kSegMax - 1) * minrows - 1) / ((kSegMax - 1) * minrows);
+  L.P = (int)(((pmin + kAttendWave - 1) / kAttendWave) * kAttendWave);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t o = off;
@@ -110,8 +113,8 @@ Layout layout(const hardkv_desc *d) {
   };
   L.scores = take(U * R * 4);
   L.tile_max = take(U * (size_t)L.tm_stride * 4);
-  L.part = take((size_t)L.P * kSegMax * G * (d->head_dim + 2) * 4);
-  L.pre = take((U + 1) * 4);
+  L.part = take((size_t)L.P * kSegMax * kAttParts * G * (d->head_dim + 2) * 4);
+  L.counters = take(U * 4);
   L.st_q = take((size_t)d->batch * d->n_q_heads * d->head_dim * e);
   L.st_k = take(U * d->head_dim * e);
   L.st_v = take(U * d->head_dim * e);
@@ -182,7 +185,9 @@ int device_sms() {
 // calls (for instance during stream capture) only read the cache.
 template <typename K>
 int set_smem(K kernel, size_t bytes) {
-  if (bytes <= 48 * 1024) return HARDKV_OK;
+  // static + dynamic shared memory above 48 KB needs the attribute, so raise it for any
+  // dynamic size (once)
+  if (bytes == 0) return HARDKV_OK;
   struct Entry {
     const void *fn;
     int dev;
@@ -272,13 +277,14 @@ int resident_ctas(K kernel, int threads, size_t smem) {
 }
 
 int launch_append(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *k_new,
-                  const void *v_new, cudaStream_t st) {
+                  const void *v_new, void *ws, const Layout &L, cudaStream_t st) {
+  int *counters = reinterpret_cast<int *>(static_cast<char *>(ws) + L.counters);
   if (d->dtype == HARDKV_BF16)
     append_kernel<bf16><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const bf16 *>(k_new),
-                                              static_cast<const bf16 *>(v_new));
+                                              static_cast<const bf16 *>(v_new), counters);
   else
     append_kernel<float><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const float *>(k_new),
-                                               static_cast<const float *>(v_new));
+                                               static_cast<const float *>(v_new), counters);
   HKV_CHECK_LAUNCH("append_kernel");
   return HARDKV_OK;
 }
@@ -298,17 +304,17 @@ int launch_condense(const hardkv_desc *d, const Shape &sh, const Cache &c, cudaS
   return HARDKV_OK;
 }
 
-template <int D>
+template <int D, int NT>
 int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
                      float *scores, float *tm, int tm_stride, int select_mode, cudaStream_t st) {
   CUtensorMap map;
   HKV_TRY(make_kmap(&map, d, c.k_ring));
   const size_t smem = ScoreTma<D>::smem_bytes(sh.B);
-  HKV_TRY(set_smem(score_tma_kernel<D>, smem));
+  HKV_TRY(set_smem(score_tma_kernel<D, NT>, smem));
   static int per_sm = 0;
-  if (!per_sm) per_sm = resident_ctas(score_tma_kernel<D>, ScoreTma<D>::THREADS, smem);
+  if (!per_sm) per_sm = resident_ctas(score_tma_kernel<D, NT>, ScoreTma<D>::THREADS, smem);
   const int grid = per_sm * device_sms();
-  score_tma_kernel<D><<<grid, ScoreTma<D>::THREADS, smem, st>>>(
+  score_tma_kernel<D, NT><<<grid, ScoreTma<D>::THREADS, smem, st>>>(
       sh, c, static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
   HKV_CHECK_LAUNCH("score_tma_kernel");
   return HARDKV_OK;
@@ -319,8 +325,11 @@ int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const vo
   float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + L.scores);
   float *tm = reinterpret_cast<float *>(static_cast<char *>(ws) + L.tile_max);
   if (d->dtype == HARDKV_BF16) {
-    return sh.d == 128 ? launch_score_tma<128>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
-                       : launch_score_tma<64>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
+    if (sh.G <= 8)
+      return sh.d == 128 ? launch_score_tma<128, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
+                         : launch_score_tma<64, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
+    return sh.d == 128 ? launch_score_tma<128, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
+                       : launch_score_tma<64, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
   }
   const dim3 grid(sh.R / kTile + 2, sh.B * sh.H);
   score_f32_kernel<<<grid, 128, (size_t)sh.G * sh.d * 4, st>>>(
@@ -334,49 +343,65 @@ int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, cons
                 float p, int select_mode, uint32_t *mask, cudaStream_t st) {
   const float *scores = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.scores);
   const float *tm = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.tile_max);
-  topp_kernel<WRITE_IDX><<<sh.B * sh.H, kSelThreads, 0, st>>>(sh, c, scores, tm, L.tm_stride, tau, p,
-                                                             select_mode, mask);
+  // the unit's scores are cached in shared memory when a whole ring fits
+  const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
+  const size_t smem = topp_smem_bytes(cache_n);
+  HKV_TRY(set_smem(topp_kernel<WRITE_IDX>, smem));
+  topp_kernel<WRITE_IDX><<<sh.B * sh.H, kSelThreads, smem, st>>>(sh, c, scores, tm, L.tm_stride, tau,
+                                                                p, select_mode, mask, cache_n);
   HKV_CHECK_LAUNCH("topp_kernel");
   return HARDKV_OK;
 }
 
-template <typename T, int D>
-int launch_attend_t(const Shape &sh, const Cache &c, const void *q, void *ws, const Layout &L,
-                    int fused, int select_mode, cudaStream_t st) {
+AttendParams attend_params(const Shape &sh, const void *q, float *out, void *ws, const Layout &L,
+                           int fused, int select_mode) {
   AttendParams ap;
   ap.q = q;
   ap.part = reinterpret_cast<float *>(static_cast<char *>(ws) + L.part);
-  ap.pre_out = reinterpret_cast<int *>(static_cast<char *>(ws) + L.pre);
+  ap.counters = reinterpret_cast<int *>(static_cast<char *>(ws) + L.counters);
+  ap.out = out;
   ap.fused = fused;
   ap.select_mode = select_mode;
   ap.U = sh.B * sh.H;
   ap.P = L.P;
-  const size_t smem = AttCfg<T, D>::smem_bytes(ap.U);
-  HKV_TRY(set_smem(attend_kernel<T, D>, smem));
-  attend_kernel<T, D><<<L.P, kAttThreads, smem, st>>>(sh, c, ap);
-  HKV_CHECK_LAUNCH("attend_kernel");
+  return ap;
+}
+
+template <int D, int NT>
+int launch_attend_bulk(const Shape &sh, const Cache &c, const AttendParams &ap, cudaStream_t st) {
+  const size_t smem = BulkCfg<D>::smem_bytes(ap.U);
+  HKV_TRY(set_smem(attend_bulk_kernel<D, NT>, smem));
+  attend_bulk_kernel<D, NT><<<ap.P, kBulkThreads, smem, st>>>(sh, c, ap);
+  HKV_CHECK_LAUNCH("attend_bulk_kernel");
   return HARDKV_OK;
 }
 
-int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, void *ws,
-                  const Layout &L, int fused, int select_mode, cudaStream_t st) {
-  if (d->dtype == HARDKV_BF16)
-    return sh.d == 128 ? launch_attend_t<bf16, 128>(sh, c, q, ws, L, fused, select_mode, st)
-                       : launch_attend_t<bf16, 64>(sh, c, q, ws, L, fused, select_mode, st);
-  return sh.d == 128 ? launch_attend_t<float, 128>(sh, c, q, ws, L, fused, select_mode, st)
-                     : launch_attend_t<float, 64>(sh, c, q, ws, L, fused, select_mode, st);
+template <int D>
+int launch_attend_f32(const Shape &sh, const Cache &c, const AttendParams &ap, cudaStream_t st) {
+  const size_t smem = F32Cfg<D>::smem_bytes(ap.U);
+  HKV_TRY(set_smem(attend_f32_kernel<D>, smem));
+  attend_f32_kernel<D><<<ap.P, kF32Threads, smem, st>>>(sh, c, ap);
+  HKV_CHECK_LAUNCH("attend_f32_kernel");
+  return HARDKV_OK;
 }
 
-int launch_combine(const Shape &sh, void *ws, const Layout &L, float *out, cudaStream_t st) {
-  const float *part = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.part);
-  const int *pre = reinterpret_cast<const int *>(static_cast<char *>(ws) + L.pre);
-  const int U = sh.B * sh.H;
-  if (sh.d == 128)
-    combine_kernel<128><<<U, 128, 0, st>>>(sh, part, pre, U, L.P, out);
-  else
-    combine_kernel<64><<<U, 64, 0, st>>>(sh, part, pre, U, L.P, out);
-  HKV_CHECK_LAUNCH("combine_kernel");
-  return HARDKV_OK;
+// Split-K attention + in-kernel combine. The per-unit completion counters must be zero
+// at launch: the fused step's append kernel zeroes them; otherwise a memset does.
+int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, float *out,
+                  void *ws, const Layout &L, int fused, int select_mode, bool zero_counters,
+                  cudaStream_t st) {
+  if (zero_counters) {
+    cudaError_t e = cudaMemsetAsync(static_cast<char *>(ws) + L.counters, 0,
+                                    (size_t)sh.B * sh.H * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  }
+  const AttendParams ap = attend_params(sh, q, out, ws, L, fused, select_mode);
+  if (d->dtype == HARDKV_BF16) {
+    if (sh.G <= 8)
+      return sh.d == 128 ? launch_attend_bulk<128, 1>(sh, c, ap, st) : launch_attend_bulk<64, 1>(sh, c, ap, st);
+    return sh.d == 128 ? launch_attend_bulk<128, 2>(sh, c, ap, st) : launch_attend_bulk<64, 2>(sh, c, ap, st);
+  }
+  return sh.d == 128 ? launch_attend_f32<128>(sh, c, ap, st) : launch_attend_f32<64>(sh, c, ap, st);
 }
 
 int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const uint32_t *mask,
@@ -418,7 +443,8 @@ int hardkv_append(const hardkv_desc *desc, const hardkv_cache *cache, const void
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_ptr(k_new));
   HKV_TRY(check_ptr(v_new));
-  return launch_append(desc, make_shape(desc), make_cache(cache), k_new, v_new, stream);
+  return launch_append(desc, make_shape(desc), make_cache(cache), k_new, v_new, ws, layout(desc),
+                       stream);
 }
 
 int hardkv_condense(const hardkv_desc *desc, const hardkv_cache *cache, void *ws,
@@ -458,8 +484,8 @@ int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const
   HKV_TRY(check_ptr(out));
   const Shape sh = make_shape(desc);
   const Layout L = layout(desc);
-  HKV_TRY(launch_attend(desc, sh, make_cache(cache), q, ws, L, 0, HARDKV_SELECT_ALL, stream));
-  return launch_combine(sh, ws, L, out, stream);
+  return launch_attend(desc, sh, make_cache(cache), q, out, ws, L, 0, HARDKV_SELECT_ALL, true,
+                       stream);
 }
 
 int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
@@ -479,7 +505,7 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   const Layout L = layout(desc);
   cudaEvent_t *ev = a->stage_events;
   HKV_TRY(record(ev, 0, stream));
-  HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, stream));
+  HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, ws, L, stream));  // zeroes counters
   HKV_TRY(record(ev, 1, stream));
   HKV_TRY(launch_condense(desc, sh, c, stream));
   HKV_TRY(record(ev, 2, stream));
@@ -487,10 +513,8 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(record(ev, 3, stream));
   HKV_TRY(launch_topp<true>(sh, c, ws, L, a->tau, a->p, a->select_mode, a->mask, stream));
   HKV_TRY(record(ev, 4, stream));
-  HKV_TRY(launch_attend(desc, sh, c, a->q, ws, L, 1, a->select_mode, stream));
-  HKV_TRY(record(ev, 5, stream));
-  HKV_TRY(launch_combine(sh, ws, L, a->out, stream));
-  return record(ev, 6, stream);
+  HKV_TRY(launch_attend(desc, sh, c, a->q, a->out, ws, L, 1, a->select_mode, false, stream));
+  return record(ev, 5, stream);
 }
 
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,

@@ -3,9 +3,10 @@
 //
 // bf16 path: a persistent kernel streams 64-row key tiles of every selected unit's
 // Sparse range with TMA (2-D tensor map over the ring, 128-byte swizzle) into a
-// multi-stage mbarrier pipeline; four consumer warps each take 16 rows of a tile and
-// compute the (query x key) logits with mma.sync m16n8k16 (queries in M, padded to
-// 16; keys in N), then max-pool over the real queries. Work is split evenly over all
+// multi-stage mbarrier pipeline; two groups of four consumer warps take alternate
+// tiles, each warp 16 rows of a tile, and compute the (key x query) logits with
+// mma.sync m16n8k16 (keys in M, queries in N, one or two 8-query tiles), then max-pool
+// over the real queries. Work is split evenly over all
 // tiles of all units, so ragged sequence lengths stay balanced.
 #pragma once
 #include "common.cuh"
@@ -21,10 +22,14 @@ struct ScoreTma {
   static constexpr int BOX_BYTES = kTile * 128;  // 64 rows x 128 bytes
   static constexpr int TILE_BYTES = BOXES * BOX_BYTES;
   static constexpr int STAGES = D == 128 ? 6 : 10;
-  static constexpr int CONSUMER_WARPS = 4;
+  static constexpr int CONSUMER_WARPS = 8;  // two groups of 4 warps on alternating tiles
+  static constexpr int GROUP_WARPS = 4;     // warps sharing one tile (16 rows each)
   static constexpr int THREADS = 32 * (CONSUMER_WARPS + 1);
+  // a stage is always refilled for the same consumer group (tile i -> stage i % STAGES,
+  // group i % 2), so each group sees every phase of its stages' barriers
+  static_assert(STAGES % 2 == 0, "stages must be even");
   static size_t smem_bytes(int B) {
-    return (size_t)STAGES * TILE_BYTES + 1024 + 2 * STAGES * 8 + 16 + (size_t)(3 * B + 1) * 4;
+    return (size_t)STAGES * TILE_BYTES + 1024 + 2 * STAGES * 8 + 16 + (size_t)(5 * B + 1) * 4;
   }
 };
 
@@ -41,24 +46,26 @@ __device__ __forceinline__ TileSpan tile_span(const Bounds &bd) {
   return t;
 }
 
-// Loads query fragments (A operand, queries in M) of unit (b,h) for all k-steps.
-template <int D>
-__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[D / 16][4], const bf16 *q, int b,
-                                             int h, const Shape &sh, int lane) {
+// Q^T fragments of unit (b,h) as the B operand (channels in K, queries in N; NT query
+// tiles of 8), for all channel steps; queries past the group are zero.
+template <int D, int NT>
+__device__ __forceinline__ void load_qT_frags(uint32_t (&qb)[NT][D / 16][2], const bf16 *q, int b, int h,
+                                              const Shape &sh, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const bf16 *q0 = q + ((size_t)b * sh.Hq + (size_t)h * sh.G) * D;
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
+  for (int nt = 0; nt < NT; ++nt) {
+    const int qi = nt * 8 + g;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int qi = g + ((r & 1) << 3);
-      const int ch = kk * 16 + ((r >> 1) << 3) + 2 * t;
-      qa[kk][r] = qi < sh.G ? *reinterpret_cast<const uint32_t *>(q0 + (size_t)qi * D + ch) : 0u;
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const int ch = kk * 16 + 2 * t;
+      qb[nt][kk][0] = qi < sh.G ? *reinterpret_cast<const uint32_t *>(q0 + (size_t)qi * D + ch) : 0u;
+      qb[nt][kk][1] = qi < sh.G ? *reinterpret_cast<const uint32_t *>(q0 + (size_t)qi * D + ch + 8) : 0u;
     }
   }
 }
 
-template <int D>
+template <int D, int NT>
 __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
     score_tma_kernel(Shape sh, Cache c, const bf16 *__restrict__ q, float *__restrict__ scores,
                      float *__restrict__ tile_max, int tm_stride, int select_mode,
@@ -73,12 +80,14 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
   int *pre = abort_flag + 4;        // [B+1] tile prefix
   int *first = pre + sh.B + 1;      // [B]
   int *ntile = first + sh.B;        // [B]
+  int *slo_s = ntile + sh.B;        // [B] Sparse range of each sequence
+  int *dlo_s = slo_s + sh.B;        // [B]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], Cfg::CONSUMER_WARPS);
+      mbar_init(&empty[s], Cfg::GROUP_WARPS);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -91,9 +100,12 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
       int v = 0;
       if (b < sh.B) {
         TileSpan ts{0, 0};
-        if (unit_active(select_mode, c.moved, b)) ts = tile_span(load_bounds(c, b, sh.R));
+        const Bounds bd = load_bounds(c, b, sh.R);
+        if (unit_active(select_mode, c.moved, b)) ts = tile_span(bd);
         first[b] = ts.first;
         ntile[b] = ts.n;
+        slo_s[b] = bd.s_lo;
+        dlo_s[b] = bd.d_lo;
         v = ts.n * sh.H;
       }
       int incl = v;
@@ -144,18 +156,21 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
     return;
   }
 
-  // ---------------- consumers: warp w takes rows [16w, 16w+16) of every tile
+  // ---------------- consumers: group k takes tiles i with i % 2 == k; warp wg of a
+  // group takes rows [16 wg, 16 wg + 16) of its tiles
   const int g = lane >> 2, t = lane & 3;
-  uint32_t qa[D / 16][4];
+  const int group = warp / Cfg::GROUP_WARPS, wg = warp % Cfg::GROUP_WARPS;
+  uint32_t qb[NT][D / 16][2];
   int cur_u = -1, b = 0;
   long long i = 0;
   for (long long gg = g0; gg < g1; ++gg, ++i) {
     while (gg >= pre[b + 1]) ++b;
     const int idx = (int)(gg - pre[b]);
+    if ((int)(i & 1) != group) continue;
     const int h = idx / ntile[b], lt = idx % ntile[b];
     const int u = b * sh.H + h;
     if (u != cur_u) {
-      load_q_frags<D>(qa, q, b, h, sh, lane);
+      load_qT_frags<D, NT>(qb, q, b, h, sh, lane);
       cur_u = u;
     }
     const int st = (int)(i % Cfg::STAGES);
@@ -164,43 +179,63 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
       flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
       break;
     }
+    // S^T for 16 key rows (keys in M, queries in N): two accumulation chains
     const uint32_t base = smem_u32(tiles + st * Cfg::TILE_BYTES);
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    const int r = warp * 16 + (lane & 7) + (((lane >> 4) & 1) << 3);
+    float sa[NT][4], sb[NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sa[nt][e] = sb[nt][e] = 0.f;
+    const int jq = lane >> 3;
+    const int r = wg * 16 + (lane & 7) + ((jq & 1) << 3);
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
-      const int ch = kk * 16 + (((lane >> 3) & 1) << 3);
+      const int ch = kk * 16 + ((jq >> 1) << 3);
       const uint32_t addr = base + (ch >> 6) * Cfg::BOX_BYTES + swz128(r, (ch & 63) >> 3);
-      uint32_t b0, b1, b2, b3;
-      ldsm_x4(b0, b1, b2, b3, addr);
-      mma_bf16(acc[0], qa[kk], b0, b1);
-      mma_bf16(acc[1], qa[kk], b2, b3);
+      uint32_t a[4];
+      ldsm_x4(a[0], a[1], a[2], a[3], addr);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (kk & 1)
+          mma_bf16(sb[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+        else
+          mma_bf16(sa[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
+      }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
 
-    // max-pool over the real queries (rows g and g+8 of M)
-    const Bounds bd{c.len[b], c.d_lo[b], c.s_lo[b], true};
-    const long long pbase = (long long)(first[b] + lt) * kTile + warp * 16;
-    float tmax = -INFINITY;
+    // max-pool over the real queries: key rows g (entries 0,1) and g+8 (entries 2,3)
+    const int s_lo = slo_s[b], d_lo = dlo_s[b];
+    const long long pbase = (long long)(first[b] + lt) * kTile + wg * 16;
+    float v0 = -INFINITY, v8 = -INFINITY;
 #pragma unroll
-    for (int n = 0; n < 2; ++n) {
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        float v = fmaxf(g < sh.G ? acc[n][e] : -INFINITY, g + 8 < sh.G ? acc[n][2 + e] : -INFINITY);
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 16));
-        const long long pos = pbase + n * 8 + 2 * t + e;
-        if (lane < 4 && pos >= bd.s_lo && pos < bd.d_lo) {
-          const float s = v * sh.scale;
-          scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
+        if (nt * 8 + 2 * t + e < sh.G) {
+          v0 = fmaxf(v0, sa[nt][e] + sb[nt][e]);
+          v8 = fmaxf(v8, sa[nt][2 + e] + sb[nt][2 + e]);
+        }
+      }
+    v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, 1));
+    v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, 2));
+    v8 = fmaxf(v8, __shfl_xor_sync(0xffffffffu, v8, 1));
+    v8 = fmaxf(v8, __shfl_xor_sync(0xffffffffu, v8, 2));
+    float tmax = -INFINITY;
+    if (t == 0) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        const long long pos = pbase + g + 8 * hr;
+        if (pos >= s_lo && pos < d_lo) {
+          const float s = (hr ? v8 : v0) * sh.scale;
+          scores[(size_t)u * sh.R + (size_t)(pos - s_lo)] = s;
           tmax = fmaxf(tmax, s);
         }
       }
     }
     tmax = warp_max(tmax);
-    if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + warp] = tmax;
+    if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + wg] = tmax;
   }
 }
 

@@ -10,8 +10,11 @@ namespace hardkv {
 // Copies k_new/v_new [B,H,d] into ring row len mod R, then advances the boundaries.
 template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T *k_new,
-                                                     const T *v_new) {
+                                                     const T *v_new, int *counters) {
   const int b = blockIdx.x;
+  // attention completion counters of this sequence's units start the step at zero
+  if (counters)
+    for (int h = threadIdx.x; h < sh.H; h += blockDim.x) counters[b * sh.H + h] = 0;
   const Bounds bd = load_bounds(c, b, sh.R);
   const int pos = bd.len;
   // after the write the live span [s_lo, pos] must still fit in R rows

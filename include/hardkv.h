@@ -125,7 +125,7 @@ typedef struct {
   cudaEvent_t *stage_events;/* NULL, or HARDKV_STEP_EVENTS events recorded before the
                                first stage and after each stage (capture-safe) */
 } hardkv_step_args;
-#define HARDKV_STEP_EVENTS 7  /* start, append, condense, score, topp, attend, combine */
+#define HARDKV_STEP_EVENTS 6  /* start, append, condense, score, topp, attend */
 
 /* Bytes of scratch the library needs for this descriptor (caller allocates; the
  * content need not be initialised and is not read across calls except as noted). */
