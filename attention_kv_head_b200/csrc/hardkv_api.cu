@@ -5,10 +5,11 @@
 #include <string.h>
 
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "k_attend.cuh"
-#include "k_attend_bulk.cuh"
+#include "k_attend_ws.cuh"
 #include "k_score.cuh"
 #include "k_select.cuh"
 #include "k_state.cuh"
@@ -37,7 +38,7 @@ int cuda_fail(cudaError_t e, const char *what) {
     if (r_ != HARDKV_OK) return r_; \
   } while (0)
 
-constexpr int kAttendWave = 296;  // 2 resident attend CTAs x 148 SMs on B200
+constexpr int kAttendWave = 444;  // 3 resident attend CTAs x 148 SMs on B200
 constexpr size_t kMaxSmem = 227 * 1024;
 constexpr int kToppCacheMax = 40960;  // fp32 scores cached per top-p CTA (160 KB)
 
@@ -98,8 +99,8 @@ Layout layout(const hardkv_desc *d) {
   const size_t U = (size_t)d->batch * d->n_kv_heads, R = d->ring_rows, e = elem_size(d);
   const int G = d->n_q_heads / d->n_kv_heads;
   L.tm_stride = kPartsPerTile * (d->ring_rows / kTile + 2);
-  const long long rows_max =
-      (long long)U * (d->sparse_cap + d->dense_window + d->block + d->condensed_slots);
+  const long long rows_max =  // total partition cost (gathered rows count twice)
+      (long long)U * (2ll * d->sparse_cap + d->dense_window + d->block + d->condensed_slots);
   // every unit has >= W + C rows, so a CTA range of <= (kSegMax - 1) (W + C) rows meets
   // at most kSegMax units; P is that bound rounded up to whole waves
   const long long minrows = d->dense_window + d->condensed_slots;
@@ -113,7 +114,7 @@ Layout layout(const hardkv_desc *d) {
   };
   L.scores = take(U * R * 4);
   L.tile_max = take(U * (size_t)L.tm_stride * 4);
-  L.part = take((size_t)L.P * kSegMax * kAttParts * G * (d->head_dim + 2) * 4);
+  L.part = take((size_t)L.P * kSegMax * G * (d->head_dim + kPartO) * 4);
   L.counters = take(U * 4);
   L.st_q = take((size_t)d->batch * d->n_q_heads * d->head_dim * e);
   L.st_k = take(U * d->head_dim * e);
@@ -183,6 +184,25 @@ int device_sms() {
 
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel, size); later
 // calls (for instance during stream capture) only read the cache.
+// Launches `kernel` allowing programmatic dependent launch: it may start while the
+// previous kernel on the stream finishes; every kernel of the library calls
+// griddepcontrol.wait before it reads anything an earlier kernel writes.
+template <typename... Exp, typename... Act>
+cudaError_t launch_pdl(void (*kernel)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Act &&...args) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Act>(args)...);
+}
+
 template <typename K>
 int set_smem(K kernel, size_t bytes) {
   // static + dynamic shared memory above 48 KB needs the attribute, so raise it for any
@@ -295,10 +315,10 @@ int launch_condense(const hardkv_desc *d, const Shape &sh, const Cache &c, cudaS
   const int U = sh.B * sh.H;
   if (d->dtype == HARDKV_BF16) {
     HKV_TRY(set_smem(condense_kernel<bf16>, smem));
-    condense_kernel<bf16><<<U, kCondenseThreads, smem, st>>>(sh, c);
+    launch_pdl(condense_kernel<bf16>, dim3(U), dim3(kCondenseThreads), smem, st, sh, c);
   } else {
     HKV_TRY(set_smem(condense_kernel<float>, smem));
-    condense_kernel<float><<<U, kCondenseThreads, smem, st>>>(sh, c);
+    launch_pdl(condense_kernel<float>, dim3(U), dim3(kCondenseThreads), smem, st, sh, c);
   }
   HKV_CHECK_LAUNCH("condense_kernel");
   return HARDKV_OK;
@@ -314,8 +334,8 @@ int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, cons
   static int per_sm = 0;
   if (!per_sm) per_sm = resident_ctas(score_tma_kernel<D, NT>, ScoreTma<D>::THREADS, smem);
   const int grid = per_sm * device_sms();
-  score_tma_kernel<D, NT><<<grid, ScoreTma<D>::THREADS, smem, st>>>(
-      sh, c, static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
+  launch_pdl(score_tma_kernel<D, NT>, dim3(grid), dim3(ScoreTma<D>::THREADS), smem, st, sh, c,
+             static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
   HKV_CHECK_LAUNCH("score_tma_kernel");
   return HARDKV_OK;
 }
@@ -332,8 +352,8 @@ int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const vo
                        : launch_score_tma<64, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
   }
   const dim3 grid(sh.R / kTile + 2, sh.B * sh.H);
-  score_f32_kernel<<<grid, 128, (size_t)sh.G * sh.d * 4, st>>>(
-      sh, c, static_cast<const float *>(q), scores, tm, L.tm_stride, select_mode);
+  launch_pdl(score_f32_kernel, grid, dim3(128), (size_t)sh.G * sh.d * 4, st, sh, c,
+             static_cast<const float *>(q), scores, tm, L.tm_stride, select_mode);
   HKV_CHECK_LAUNCH("score_f32_kernel");
   return HARDKV_OK;
 }
@@ -347,8 +367,8 @@ int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, cons
   const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
   const size_t smem = topp_smem_bytes(cache_n);
   HKV_TRY(set_smem(topp_kernel<WRITE_IDX>, smem));
-  topp_kernel<WRITE_IDX><<<sh.B * sh.H, kSelThreads, smem, st>>>(sh, c, scores, tm, L.tm_stride, tau,
-                                                                p, select_mode, mask, cache_n);
+  launch_pdl(topp_kernel<WRITE_IDX>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, scores, tm,
+             L.tm_stride, tau, p, select_mode, mask, cache_n);
   HKV_CHECK_LAUNCH("topp_kernel");
   return HARDKV_OK;
 }
@@ -368,11 +388,11 @@ AttendParams attend_params(const Shape &sh, const void *q, float *out, void *ws,
 }
 
 template <int D, int NT>
-int launch_attend_bulk(const Shape &sh, const Cache &c, const AttendParams &ap, cudaStream_t st) {
-  const size_t smem = BulkCfg<D>::smem_bytes(ap.U);
-  HKV_TRY(set_smem(attend_bulk_kernel<D, NT>, smem));
-  attend_bulk_kernel<D, NT><<<ap.P, kBulkThreads, smem, st>>>(sh, c, ap);
-  HKV_CHECK_LAUNCH("attend_bulk_kernel");
+int launch_attend_ws(const Shape &sh, const Cache &c, const AttendParams &ap, cudaStream_t st) {
+  const size_t smem = WsCfg<D>::smem_bytes(ap.U);
+  HKV_TRY(set_smem(attend_ws_kernel<D, NT>, smem));
+  launch_pdl(attend_ws_kernel<D, NT>, dim3(ap.P), dim3(kWsThreads), smem, st, sh, c, ap);
+  HKV_CHECK_LAUNCH("attend_ws_kernel");
   return HARDKV_OK;
 }
 
@@ -380,7 +400,7 @@ template <int D>
 int launch_attend_f32(const Shape &sh, const Cache &c, const AttendParams &ap, cudaStream_t st) {
   const size_t smem = F32Cfg<D>::smem_bytes(ap.U);
   HKV_TRY(set_smem(attend_f32_kernel<D>, smem));
-  attend_f32_kernel<D><<<ap.P, kF32Threads, smem, st>>>(sh, c, ap);
+  launch_pdl(attend_f32_kernel<D>, dim3(ap.P), dim3(kF32Threads), smem, st, sh, c, ap);
   HKV_CHECK_LAUNCH("attend_f32_kernel");
   return HARDKV_OK;
 }
@@ -398,8 +418,8 @@ int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const v
   const AttendParams ap = attend_params(sh, q, out, ws, L, fused, select_mode);
   if (d->dtype == HARDKV_BF16) {
     if (sh.G <= 8)
-      return sh.d == 128 ? launch_attend_bulk<128, 1>(sh, c, ap, st) : launch_attend_bulk<64, 1>(sh, c, ap, st);
-    return sh.d == 128 ? launch_attend_bulk<128, 2>(sh, c, ap, st) : launch_attend_bulk<64, 2>(sh, c, ap, st);
+      return sh.d == 128 ? launch_attend_ws<128, 1>(sh, c, ap, st) : launch_attend_ws<64, 1>(sh, c, ap, st);
+    return sh.d == 128 ? launch_attend_ws<128, 2>(sh, c, ap, st) : launch_attend_ws<64, 2>(sh, c, ap, st);
   }
   return sh.d == 128 ? launch_attend_f32<128>(sh, c, ap, st) : launch_attend_f32<64>(sh, c, ap, st);
 }
@@ -408,9 +428,9 @@ int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const 
                    int select_mode, cudaStream_t st) {
   const dim3 grid((sh.R + kSelThreads - 1) / kSelThreads, sh.B * sh.H);
   if (d->dtype == HARDKV_BF16)
-    compact_kernel<bf16><<<grid, kSelThreads, 0, st>>>(sh, c, mask, select_mode);
+    launch_pdl(compact_kernel<bf16>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode);
   else
-    compact_kernel<float><<<grid, kSelThreads, 0, st>>>(sh, c, mask, select_mode);
+    launch_pdl(compact_kernel<float>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode);
   HKV_CHECK_LAUNCH("compact_kernel");
   return HARDKV_OK;
 }

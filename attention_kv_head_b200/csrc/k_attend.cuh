@@ -1,8 +1,9 @@
 // Decode attention over the three tiers, optionally fused with Index Regularization.
 //
 // Every unit (b,h) has a union list: [compact slots 0..n) [Dense positions d_lo..len)
-// [Condensed slots 0..C). All units' lists are concatenated and cut into equal
-// contiguous ranges, one per CTA (split-K that stays balanced for ragged lengths).
+// [Condensed slots 0..C). All units' lists are concatenated and cut into contiguous
+// ranges of equal cost, one per CTA (split-K that stays balanced for ragged lengths; a
+// row gathered from the ring costs two, any other row one).
 // Each of a CTA's four compute warps leaves one log-sum-exp partial per unit segment
 // the CTA covers; the last CTA to finish a segment of a unit (an atomic count, no
 // waiting) merges that unit's partials into the output. In fused mode the compact
@@ -19,13 +20,13 @@
 namespace hardkv {
 
 constexpr int kAttRows = 64;   // rows per tile
-constexpr int kAttParts = 4;   // compute warps per CTA = partials per (CTA, segment)
+constexpr int kAttParts = 4;   // compute warps per CTA
 constexpr int kSegMax = 8;     // unit segments a CTA may cover
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct AttendParams {
   const void *q;     // [B,Hq,d]
-  float *part;       // [P][kSegMax][kAttParts][G][d+2]: m (log2 units), l, o[d]
+  float *part;       // [P][kSegMax][G][kPartRow]: m (log2 units), l, -, -, o[d] per CTA segment
   int *counters;     // [U] CTAs finished per unit; zero before the launch
   float *out;        // [B,Hq,d]
   int fused;         // 1: gather kept rows of reselected units from the ring + write compact
@@ -33,22 +34,70 @@ struct AttendParams {
   int U, P;          // units, CTAs
 };
 
+// A partial row is [m, l, pad, pad, o[0..d)]: d + 4 floats, so o is 16-byte aligned.
+constexpr int kPartO = 4;
 __device__ __forceinline__ float *partial_ptr(const AttendParams &ap, const Shape &sh, long long cta,
-                                              int seg, int part, int q) {
-  return ap.part + ((((size_t)cta * kSegMax + seg) * kAttParts + part) * sh.G + q) * (sh.d + 2);
+                                              int seg, int q) {
+  return ap.part + (((size_t)cta * kSegMax + seg) * sh.G + q) * (sh.d + kPartO);
 }
 
-// Rows of unit u in the concatenated list.
-__device__ __forceinline__ int unit_rows(const Shape &sh, const Cache &c, int u) {
+// Shared-memory staging of the four warps' online-softmax states: [warp][16][d+2].
+__device__ __forceinline__ float *warp_state_slot(float *scratch, int d, int w, int q) {
+  return scratch + ((size_t)w * 16 + q) * (d + 2);
+}
+
+// Merges the four warps' states (staged with warp_state_slot) into the CTA's partial of
+// segment `seg`. All threads of the block call it.
+template <int D>
+__device__ __forceinline__ void merge_warps(const Shape &sh, const AttendParams &ap, float *scratch, int seg) {
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < sh.G * D; idx += blockDim.x) {
+    const int qq = idx / D, ch = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kAttParts; ++w) M = fmaxf(M, warp_state_slot(scratch, D, w, qq)[0]);
+    float O = 0.f, Lsum = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kAttParts; ++w) {
+        const float *sl = warp_state_slot(scratch, D, w, qq);
+        if (sl[0] == -INFINITY) continue;
+        const float f = exp2f(sl[0] - M);
+        O = fmaf(sl[2 + ch], f, O);
+        Lsum = fmaf(sl[1], f, Lsum);
+      }
+    }
+    float *pq = partial_ptr(ap, sh, blockIdx.x, seg, qq);
+    if (ch == 0) {
+      pq[0] = M;
+      pq[1] = Lsum;
+    }
+    pq[kPartO + ch] = O;
+  }
+  __syncthreads();
+}
+
+// Cost of unit u in the concatenated list: one per row, two per row gathered from the
+// ring (read, then written to its compact slot). CTAs split the total cost evenly.
+__device__ __forceinline__ int unit_cost(const Shape &sh, const Cache &c, const AttendParams &ap, int u) {
   const int b = u / sh.H;
   const Bounds bd = load_bounds(c, b, sh.R);
   const int n = min(max(c.n_kept[u], 0), sh.cap);
-  return (bd.ok ? n + (bd.len - bd.d_lo) : 0) + sh.C;
+  const int wgt = (ap.fused && unit_active(ap.select_mode, c.moved, b)) ? 2 : 1;
+  return (bd.ok ? wgt * n + (bd.len - bd.d_lo) : 0) + sh.C;
 }
 
-// Prefix of unit_rows over all units into pre[0..U], computed by the first 128 threads;
+// First union row of a unit at cost offset `cst` (rows 0..n-1 cost `wgt` each, the rest
+// one each); monotone, so consecutive cost ranges give consecutive row ranges.
+__device__ __forceinline__ int cost_to_row(int cst, int n, int wgt) {
+  if (wgt == 1) return cst;
+  return cst <= 2 * n ? (cst + 1) / 2 : cst - n;
+}
+
+// Prefix of unit_cost over all units into pre[0..U], computed by the first 128 threads;
 // every thread of the block must call it (it synchronises the block).
-__device__ __forceinline__ void units_prefix(const Shape &sh, const Cache &c, int U, int *pre) {
+__device__ __forceinline__ void units_prefix(const Shape &sh, const Cache &c, const AttendParams &ap, int U,
+                                             int *pre) {
   constexpr int NT = 128;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   __shared__ int wsum[NT / 32];
@@ -57,7 +106,7 @@ __device__ __forceinline__ void units_prefix(const Shape &sh, const Cache &c, in
   int local = 0;
   if (tid < NT)
     for (int k = 0; k < per; ++k)
-      if (u0 + k < U) local += unit_rows(sh, c, u0 + k);
+      if (u0 + k < U) local += unit_cost(sh, c, ap, u0 + k);
   int incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -73,7 +122,7 @@ __device__ __forceinline__ void units_prefix(const Shape &sh, const Cache &c, in
     for (int k = 0; k < per; ++k) {
       if (u0 + k < U) {
         pre[u0 + k] = run;
-        run += unit_rows(sh, c, u0 + k);
+        run += unit_cost(sh, c, ap, u0 + k);
       }
     }
     if (tid == NT - 1) pre[U] = run;
@@ -93,71 +142,102 @@ __device__ __forceinline__ int upper_unit(const int *pre, int U, long long x) {
   return lo;
 }
 
-// Merges all partials of unit u (CTAs f..l of the partition, kAttParts each) into
-// out[b, h*G + g, :]. Run by `nthr` threads (warps 0..nthr/32-1) that synchronise with
-// `bar`; reads the partials through L2. `scratch` holds 32 floats.
-template <int D, class Bar>
+// Merges the partials of unit u (one per CTA f..l of the partition) into
+// out[b, h*G + g, :]. All 128 threads of the block call it; `scratch` holds
+// 32 + 256 * G floats. Scale factors exp2(m_i - M) are computed once per partial, then
+// every thread accumulates a float4 of outputs over the partials (many loads in flight).
+template <int D>
 __device__ __forceinline__ void combine_unit(const Shape &sh, const AttendParams &ap, const int *pre,
-                                             long long range, int u, float *scratch, int nthr,
-                                             Bar bar) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = nthr / 32;
+                                             long long range, int u, float *scratch) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   const int b = u / sh.H, h = u % sh.H, G = sh.G;
   const long long f = pre[u] / range, l = (pre[u + 1] - 1) / range;
-  const int n = (int)(l - f + 1) * kAttParts;
+  const int n = (int)(l - f + 1);
   const int seg_f = u - upper_unit(pre, ap.U, f * range);
-  float *Ms = scratch, *Ls = scratch + 16;
+  float *Ms = scratch, *Ls = scratch + 16, *fac = scratch + 32;  // fac: [256][G]
   auto part_of = [&](int i, int g) -> const float * {
-    const int k = i / kAttParts;
-    return partial_ptr(ap, sh, f + k, k == 0 ? seg_f : 0, i % kAttParts, g);
+    return partial_ptr(ap, sh, f + i, i == 0 ? seg_f : 0, g);
   };
   for (int g = warp; g < G; g += nw) {
     float M = -INFINITY;
     for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(part_of(i, g)));
     M = warp_max(M);
-    float Lsum = 0.f;
-    if (M != -INFINITY)
-      for (int i = lane; i < n; i += 32) {
-        const float *pq = part_of(i, g);
-        const float m = __ldcg(pq);
-        if (m != -INFINITY) Lsum = fmaf(__ldcg(pq + 1), exp2f(m - M), Lsum);
-      }
-    Lsum = warp_sum(Lsum);
     if (lane == 0) {
       Ms[g] = M;
-      Ls[g] = Lsum;
+      Ls[g] = 0.f;
     }
   }
-  bar();
-  float *o = ap.out + ((size_t)b * sh.Hq + (size_t)h * G) * D;
-  for (int idx = tid; idx < G * D; idx += nthr) {
-    const int g = idx / D, ch = idx % D;
-    const float M = Ms[g], Lsum = Ls[g];
-    float O = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll 4
-      for (int i = 0; i < n; ++i) {
-        const float *pq = part_of(i, g);
-        const float m = __ldcg(pq);
-        if (m != -INFINITY) O = fmaf(__ldcg(pq + 2 + ch), exp2f(m - M), O);
+  __syncthreads();
+  constexpr int C4 = D / 4;
+  constexpr int OUT_PER_THREAD = 16 * C4 / 128;  // G <= 16 queries, 128 threads
+  float4 acc[OUT_PER_THREAD];
+#pragma unroll
+  for (int r = 0; r < OUT_PER_THREAD; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i0 = 0; i0 < n; i0 += 256) {
+    const int ni = min(256, n - i0);
+    for (int k = tid; k < ni * G; k += blockDim.x) {
+      const int i = i0 + k / G, g = k % G;
+      const float m = __ldcg(part_of(i, g));
+      fac[k] = (m == -INFINITY || Ms[g] == -INFINITY) ? 0.f : exp2f(m - Ms[g]);
+    }
+    __syncthreads();
+    for (int g = warp; g < G; g += nw) {  // fixed summation order: reproducible
+      float ls = 0.f;
+      for (int i = lane; i < ni; i += 32) {
+        const float fv = fac[i * G + g];
+        if (fv != 0.f) ls = fmaf(__ldcg(part_of(i0 + i, g) + 1), fv, ls);
       }
+      ls = warp_sum(ls);
+      if (lane == 0) Ls[g] += ls;
     }
-    o[(size_t)g * D + ch] = Lsum > 0.f ? O / Lsum : 0.f;
+#pragma unroll
+    for (int r = 0; r < OUT_PER_THREAD; ++r) {  // outputs idx = tid + r * blockDim
+      const int idx = tid + r * (int)blockDim.x;
+      if (idx >= G * C4) continue;
+      const int g = idx / C4, c4 = idx % C4;
+      float4 a = acc[r];
+#pragma unroll 8
+      for (int i = 0; i < ni; ++i) {
+        const float fv = fac[i * G + g];
+        const float4 ov = __ldcg(reinterpret_cast<const float4 *>(part_of(i0 + i, g) + kPartO) + c4);
+        a.x = fmaf(ov.x, fv, a.x);
+        a.y = fmaf(ov.y, fv, a.y);
+        a.z = fmaf(ov.z, fv, a.z);
+        a.w = fmaf(ov.w, fv, a.w);
+      }
+      acc[r] = a;
+    }
+    __syncthreads();
   }
-  bar();
+  float *o = ap.out + ((size_t)b * sh.Hq + (size_t)h * G) * D;
+#pragma unroll
+  for (int r = 0; r < OUT_PER_THREAD; ++r) {
+    const int idx = tid + r * (int)blockDim.x;
+    if (idx >= G * C4) continue;
+    const int g = idx / C4, c4 = idx % C4;
+    const float Lsum = Ls[g];
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+    float4 a = acc[r];
+    a.x *= inv;
+    a.y *= inv;
+    a.z *= inv;
+    a.w *= inv;
+    reinterpret_cast<float4 *>(o + (size_t)g * D)[c4] = a;
+  }
+  __syncthreads();
 }
 
 // Counts a finished segment of unit u; true in the thread-block that finished last.
-// All participating threads call it after their partial stores; `bar` syncs them.
-template <class Bar>
-__device__ __forceinline__ bool last_to_finish(const AttendParams &ap, const int *pre, long long range,
-                                               int u, int *flag_smem, Bar bar) {
-  bar();
+// All threads call it after the block's partial stores.
+__device__ __forceinline__ bool last_to_finish(const AttendParams &ap, const int *pre, long long range, int u,
+                                               int *flag_smem) {
+  __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
     const long long f = pre[u] / range, l = (pre[u + 1] - 1) / range;
     *flag_smem = atomicAdd(ap.counters + u, 1) == (int)(l - f);
   }
-  bar();
+  __syncthreads();
   const bool last = *flag_smem != 0;
   if (last) __threadfence();
   return last;
@@ -267,7 +347,7 @@ struct F32Cfg {
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static size_t smem_bytes(int U) {
     return 16 + (size_t)kF32Stages * STAGE_BYTES + (size_t)kF32Stages * kAttRows * 8 +
-           (size_t)(U + 2) * 4 + 128;
+           (size_t)(U + 2) * 4;
   }
 };
 
@@ -281,12 +361,13 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
   uint32_t *codes = reinterpret_cast<uint32_t *>(tiles + kF32Stages * Cfg::STAGE_BYTES);  // [S][64]
   float *biases = reinterpret_cast<float *>(codes + kF32Stages * kAttRows);               // [S][64]
   int *pre = reinterpret_cast<int *>(biases + kF32Stages * kAttRows);                     // [U+1]
-  float *scratch = reinterpret_cast<float *>(pre + ap.U + 1);                             // [32]
+  float *scratch = reinterpret_cast<float *>(tiles);  // reused once a segment's tiles are done
   __shared__ int s_last;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int U = ap.U;
   pdl_wait();
-  units_prefix(sh, c, U, pre);
+  pdl_launch();
+  units_prefix(sh, c, ap, U, pre);
   const long long total = pre[U];
   const long long range = (total + ap.P - 1) / ap.P;
   long long start = range * blockIdx.x;
@@ -294,7 +375,6 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
   if (start >= end) return;
   int u = upper_unit(pre, U, start);
   const float *q = static_cast<const float *>(ap.q);
-  auto bar = [] { __syncthreads(); };
 
   for (int seg = 0; start < end; ++seg) {
     if (seg >= kSegMax) {
@@ -303,8 +383,9 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
     }
     const int b = u / sh.H, h = u % sh.H;
     const UnitView v = unit_view(sh, c, ap, u);
-    const int r0 = (int)(start - pre[u]);
-    const int r1 = (int)(min(end, (long long)pre[u + 1]) - pre[u]);
+    const int wgt = v.gather ? 2 : 1;
+    const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, wgt);
+    const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, wgt);
     const int ntiles = (r1 - r0 + kAttRows - 1) / kAttRows;
     const size_t rb = (size_t)D * 4;
     const uint8_t *kring = static_cast<const uint8_t *>(c.k_ring) + (size_t)u * sh.R * rb;
@@ -403,20 +484,20 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
       }
       __syncthreads();
     }
-    // this warp's partial
+    // this warp's state -> shared memory, then one partial for the CTA's segment
 #pragma unroll
     for (int g = 0; g < 16; ++g) {
       if (g >= sh.G) break;
-      float *pq = partial_ptr(ap, sh, blockIdx.x, seg, warp, g);
+      float *sl = warp_state_slot(scratch, D, warp, g);
       if (lane == 0) {
-        pq[0] = m[g];
-        pq[1] = l[g];
+        sl[0] = m[g];
+        sl[1] = l[g];
       }
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) pq[2 + lane + 32 * i] = o[g][i];
+      for (int i = 0; i < D / 32; ++i) sl[2 + lane + 32 * i] = o[g][i];
     }
-    if (last_to_finish(ap, pre, range, u, &s_last, bar))
-      combine_unit<D>(sh, ap, pre, range, u, scratch, kF32Threads, bar);
+    merge_warps<D>(sh, ap, scratch, seg);
+    if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u, scratch);
     start = pre[u + 1];
     ++u;
   }

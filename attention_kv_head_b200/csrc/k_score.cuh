@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
     fence_barrier_init();
   }
   if (warp == Cfg::CONSUMER_WARPS && lane == 0) tma_prefetch_desc(&kmap);
+  pdl_wait();  // boundaries and keys come from the previous kernels
+  pdl_launch();
   if (warp == 0) {  // per-sequence tile spans and their prefix over (b, h)
     int carry = 0;
     for (int b0 = 0; b0 < sh.B; b0 += 32) {
@@ -244,6 +246,8 @@ __global__ void __launch_bounds__(128)
     score_f32_kernel(Shape sh, Cache c, const float *__restrict__ q, float *__restrict__ scores,
                      float *__restrict__ tile_max, int tm_stride, int select_mode) {
   const int u = blockIdx.y, b = u / sh.H, h = u % sh.H;
+  pdl_wait();
+  pdl_launch();
   if (!unit_active(select_mode, c.moved, b)) return;
   const Bounds bd = load_bounds(c, b, sh.R);
   const TileSpan ts = tile_span(bd);

@@ -176,6 +176,8 @@ __global__ void __launch_bounds__(kSelThreads)
                 const float *__restrict__ tile_max, int tm_stride, const float *__restrict__ tau,
                 float p, int select_mode, uint32_t *__restrict__ mask, int cache_n) {
   const int u = blockIdx.x, b = u / sh.H;
+  pdl_wait();
+  pdl_launch();
   if (!unit_active(select_mode, c.moved, b)) return;
   __shared__ SelShared S;
   extern __shared__ unsigned long long sel_dyn[];
@@ -184,7 +186,6 @@ __global__ void __launch_bounds__(kSelThreads)
   uint32_t *ckey = hcnt + kBins;                                         // [kCandMax]
   float *score_cache = reinterpret_cast<float *>(ckey + kCandMax);      // [cache_n]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();
   const Bounds bd = load_bounds(c, b, sh.R);
   if (!bd.ok && tid == 0) flag(c.status, HARDKV_DEV_BAD_BOUNDS);
   const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
@@ -409,6 +410,8 @@ template <typename T>
 __global__ void __launch_bounds__(kSelThreads)
     compact_kernel(Shape sh, Cache c, const uint32_t *__restrict__ mask, int select_mode) {
   const int u = blockIdx.y, b = u / sh.H;
+  pdl_wait();
+  pdl_launch();
   if (!unit_active(select_mode, c.moved, b)) return;
   __shared__ int scan[40];
   __shared__ int list_slot[kSelThreads];

@@ -12,6 +12,8 @@ template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T *k_new,
                                                      const T *v_new, int *counters) {
   const int b = blockIdx.x;
+  pdl_wait();  // the previous step's kernels finish before this one touches the state
+  pdl_launch();
   // attention completion counters of this sequence's units start the step at zero
   if (counters)
     for (int h = threadIdx.x; h < sh.H; h += blockDim.x) counters[b * sh.H + h] = 0;
@@ -72,6 +74,8 @@ __host__ __device__ inline size_t condense_smem_floats(int blk, int d, int C) {
 template <typename T>
 __global__ void __launch_bounds__(kCondenseThreads) condense_kernel(Shape sh, Cache c) {
   const int u = blockIdx.x, b = u / sh.H;
+  pdl_wait();
+  pdl_launch();
   if (c.moved[b] == 0) return;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   constexpr int NW = kCondenseThreads / 32;

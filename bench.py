@@ -41,7 +41,7 @@ NOMINAL_HBM_GBS = 8000.0
 STAGES = ("append", "condense", "score", "topp", "attend")
 KERNEL_OF_STAGE = {"append": "append_kernel", "condense": "condense_kernel",
                    "score": "score_tma_kernel", "topp": "topp_kernel",
-                   "attend": "attend_bulk_kernel"}
+                   "attend": "attend_ws_kernel"}
 
 
 # ----------------------------------------------------------------------------- helpers

@@ -62,8 +62,10 @@ def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_ex
     v_sp = U.device_rows(dc.v_sp)
     o = out.cpu().numpy()
     lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
+    results = {}
     for (b, h), unit in units.items():
         res = unit.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, p)
+        results[b, h] = res
         assert (lens[b], dlo[b], slo[b]) == (unit.len, unit.d_lo, unit.s_lo)
         L = unit.d_lo - unit.s_lo
         kept = U.mask_bits(m[b, h], L)
@@ -80,6 +82,8 @@ def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_ex
         if same:
             assert n == res.n and np.array_equal(sp_idx[b, h], res.idx)
             cmp.attention(o[b, h * G:(h + 1) * G], res.out)
+        results[b, h] = (res, same)
+    return results
 
 
 @pytest.mark.parametrize("name", list(SMALL))
@@ -105,8 +109,8 @@ def test_small_step_unfused_vs_oracle_and_fused(name):
         got = sc[b * w.n_kv_heads + h, :L]
         assert np.allclose(got, ref, rtol=1e-5, atol=1e-5 * np.abs(ref).max()), name
     cmp = U.StepCompare(w.dtype)
-    compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp)
-    # fused step == unfused path, bit for bit
+    results = compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp)
+    # fused step == unfused path (selection, compaction and bookkeeping bit for bit)
     assert torch.equal(mask, mask2)
     assert torch.equal(dc.n_kept, dc2.n_kept) and torch.equal(dc.sp_idx, dc2.sp_idx)
     for t1, t2 in ((dc.len, dc2.len), (dc.d_lo, dc2.d_lo), (dc.s_lo, dc2.s_lo)):
@@ -116,7 +120,13 @@ def test_small_step_unfused_vs_oracle_and_fused(name):
         for h in range(w.n_kv_heads):
             assert torch.equal(dc.k_sp[b, h, :n[b, h]], dc2.k_sp[b, h, :n[b, h]])
             assert torch.equal(dc.v_sp[b, h, :n[b, h]], dc2.v_sp[b, h, :n[b, h]])
-    assert torch.equal(out, out2)
+    # the fused path splits the work by cost (gathered rows weigh two), the standalone
+    # attention by rows: same math, different split-K summation order, so the fused
+    # output is held to the oracle bound itself
+    o2 = out2.cpu().numpy()
+    for (b, h), (res, same) in results.items():
+        if same:
+            cmp.attention(o2[b, h * w.group:(h + 1) * w.group], res.out)
     st_words = dc.read_status()
     assert st_words[B.ST_FLAGS] == 0
     assert st_words[B.ST_SELECTIONS] == w.units
