@@ -76,17 +76,22 @@ def normal(key: int, start: int, count: int) -> np.ndarray:
     """`count` N(0,1) float64 draws, elements [start, start+count) of stream `key`.
 
     Element i uses Box-Muller pair i//2 (cos for even i, sin for odd i); the pair's
-    two uniforms are splitmix64 outputs 2m and 2m+1 of the stream.
+    two uniforms are splitmix64 outputs 2m and 2m+1 of the stream. Each pair is
+    evaluated once and both of its draws are kept.
     """
     if count <= 0:
         return np.zeros(0, np.float64)
-    i = np.arange(start, start + count, dtype=np.uint64)
-    m = i >> np.uint64(1)
+    m0, m1 = start >> 1, (start + count - 1) >> 1
+    m = np.arange(m0, m1 + 1, dtype=np.uint64)
     u1 = uniform(key, m * np.uint64(2))
     u2 = uniform(key, m * np.uint64(2) + np.uint64(1))
     r = np.sqrt(-2.0 * np.log(u1))
     th = 2.0 * math.pi * u2
-    return np.where((i & np.uint64(1)) == 0, r * np.cos(th), r * np.sin(th))
+    pairs = np.empty((m.size, 2), np.float64)
+    pairs[:, 0] = r * np.cos(th)
+    pairs[:, 1] = r * np.sin(th)
+    off = start - 2 * m0
+    return pairs.reshape(-1)[off:off + count]
 
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
