@@ -46,6 +46,12 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 size_t elem_size(const hardkv_desc *d) { return d->dtype == HARDKV_BF16 ? 2 : 4; }
 
+// Largest attention-partition cost of one unit (see unit_cost).
+long long unit_cost_max(const hardkv_desc *d) {
+  return kSegCost + (long long)kCostGather * d->sparse_cap +
+         (long long)kCostRow * (d->dense_window + d->block + d->condensed_slots);
+}
+
 int validate_desc(const hardkv_desc *d) {
   if (!d) return HARDKV_EINVAL;
   if (d->dtype != HARDKV_F32 && d->dtype != HARDKV_BF16) return HARDKV_EDTYPE;
@@ -61,8 +67,13 @@ int validate_desc(const hardkv_desc *d) {
   if (d->condense_mode != HARDKV_EVICT && d->condense_mode != HARDKV_MERGE) return HARDKV_EINVAL;
   if (d->sparse_cap < 1) return HARDKV_ECAP;
   if (d->ring_rows % 64 != 0 || d->ring_rows < d->dense_window + d->block) return HARDKV_ECAP;
+  if (d->ring_rows > kMaxSelectRows) return HARDKV_EINVAL;
   const long long U = (long long)d->batch * d->n_kv_heads;
   if (U * d->ring_rows >= (1ll << 31) || U * d->sparse_cap >= (1ll << 31)) return HARDKV_EINVAL;
+  // the attention partition's prefix sums are 32-bit (a Dense span is at most R rows)
+  if (U * (kSegCost + (long long)kCostGather * d->sparse_cap +
+           (long long)kCostRow * (d->ring_rows + d->condensed_slots)) >= (1ll << 31))
+    return HARDKV_EINVAL;
   if (d->condense_mode == HARDKV_MERGE &&
       (d->condensed_slots > 2048 ||
        condense_smem_floats(d->block, d->head_dim, d->condensed_slots) * 4 > kMaxSmem))
@@ -99,12 +110,12 @@ Layout layout(const hardkv_desc *d) {
   const size_t U = (size_t)d->batch * d->n_kv_heads, R = d->ring_rows, e = elem_size(d);
   const int G = d->n_q_heads / d->n_kv_heads;
   L.tm_stride = kPartsPerTile * (d->ring_rows / kTile + 2);
-  const long long rows_max =  // total partition cost (gathered rows count twice)
-      (long long)U * (2ll * d->sparse_cap + d->dense_window + d->block + d->condensed_slots);
-  // every unit has >= W + C rows, so a CTA range of <= (kSegMax - 1) (W + C) rows meets
-  // at most kSegMax units; P is that bound rounded up to whole waves
-  const long long minrows = d->dense_window + d->condensed_slots;
-  const long long pmin = (rows_max + (kSegMax - 1) * minrows - 1) / ((kSegMax - 1) * minrows);
+  const long long cost_max = (long long)U * unit_cost_max(d);  // total partition cost
+  // every unit costs >= kSegCost + kCostRow (W + C), so a CTA range of at most
+  // (kSegMax - 1) times that meets at most kSegMax units; P is that bound rounded up to
+  // whole waves
+  const long long minc = kSegCost + (long long)kCostRow * (d->dense_window + d->condensed_slots);
+  const long long pmin = (cost_max + (kSegMax - 1) * minc - 1) / ((kSegMax - 1) * minc);
   L.P = (int)(((pmin + kAttendWave - 1) / kAttendWave) * kAttendWave);
   size_t off = 0;
   auto take = [&](size_t bytes) {

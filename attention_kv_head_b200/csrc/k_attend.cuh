@@ -3,7 +3,7 @@
 // Every unit (b,h) has a union list: [compact slots 0..n) [Dense positions d_lo..len)
 // [Condensed slots 0..C). All units' lists are concatenated and cut into contiguous
 // ranges of equal cost, one per CTA (split-K that stays balanced for ragged lengths; a
-// row gathered from the ring costs two, any other row one).
+// row gathered from the ring costs 3, any other row 2, each unit segment 320).
 // Each of a CTA's four compute warps leaves one log-sum-exp partial per unit segment
 // the CTA covers; the last CTA to finish a segment of a unit (an atomic count, no
 // waiting) merges that unit's partials into the output. In fused mode the compact
@@ -12,7 +12,7 @@
 // summary sec. 2.C Rewrite Cache), so kept rows are read once.
 //
 // This file: the shared partition / row / combine code and the fp32 kernel (cp.async
-// staging, CUDA-core FMA). The bf16 kernel is in k_attend_bulk.cuh.
+// staging, CUDA-core FMA). The bf16 kernel is in k_attend_ws.cuh.
 #pragma once
 #include "common.cuh"
 #include "k_score.cuh"
@@ -77,21 +77,29 @@ __device__ __forceinline__ void merge_warps(const Shape &sh, const AttendParams 
   __syncthreads();
 }
 
-// Cost of unit u in the concatenated list: one per row, two per row gathered from the
-// ring (read, then written to its compact slot). CTAs split the total cost evenly.
+// Partition cost of unit u: kSegCost for the segment it opens in some CTA (q load,
+// pipeline fill, partial store, count), then kCostGather per compact row gathered from
+// the ring (read, then written to its compact slot) and kCostRow per other row. The
+// weights follow measured per-row times of the bf16 kernel on B200 (about 55 ns per
+// gathered row and 37 ns per contiguous row per CTA, 6-9 us per extra segment).
+constexpr int kCostRow = 2, kCostGather = 3, kSegCost = 320;
+
 __device__ __forceinline__ int unit_cost(const Shape &sh, const Cache &c, const AttendParams &ap, int u) {
   const int b = u / sh.H;
   const Bounds bd = load_bounds(c, b, sh.R);
   const int n = min(max(c.n_kept[u], 0), sh.cap);
-  const int wgt = (ap.fused && unit_active(ap.select_mode, c.moved, b)) ? 2 : 1;
-  return (bd.ok ? wgt * n + (bd.len - bd.d_lo) : 0) + sh.C;
+  const int wgt = (ap.fused && unit_active(ap.select_mode, c.moved, b)) ? kCostGather : kCostRow;
+  return kSegCost + (bd.ok ? wgt * n + kCostRow * (bd.len - bd.d_lo) : 0) + kCostRow * sh.C;
 }
 
-// First union row of a unit at cost offset `cst` (rows 0..n-1 cost `wgt` each, the rest
-// one each); monotone, so consecutive cost ranges give consecutive row ranges.
+// Union rows of a unit that start before cost offset `cst` (the first kSegCost is the
+// segment overhead; rows 0..n-1 cost `wgt` each, the rest kCostRow each). Monotone, so
+// consecutive cost ranges give consecutive, disjoint row ranges.
 __device__ __forceinline__ int cost_to_row(int cst, int n, int wgt) {
-  if (wgt == 1) return cst;
-  return cst <= 2 * n ? (cst + 1) / 2 : cst - n;
+  const int x = cst - kSegCost;
+  if (x <= 0) return 0;
+  if (x <= wgt * n) return (x + wgt - 1) / wgt;
+  return n + (x - wgt * n + kCostRow - 1) / kCostRow;
 }
 
 // Prefix of unit_cost over all units into pre[0..U], computed by the first 128 threads;
@@ -143,88 +151,74 @@ __device__ __forceinline__ int upper_unit(const int *pre, int U, long long x) {
 }
 
 // Merges the partials of unit u (one per CTA f..l of the partition) into
-// out[b, h*G + g, :]. All 128 threads of the block call it; `scratch` holds
-// 32 + 256 * G floats. Scale factors exp2(m_i - M) are computed once per partial, then
-// every thread accumulates a float4 of outputs over the partials (many loads in flight).
+// out[b, h*G + g, :]. Each thread owns float4 outputs (g, c4) and folds the partials in
+// CTA order with a running max: one L2 round trip per 8 partials, no shared memory, no
+// block barrier, and a fixed order (reproducible).
 template <int D>
 __device__ __forceinline__ void combine_unit(const Shape &sh, const AttendParams &ap, const int *pre,
-                                             long long range, int u, float *scratch) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+                                             long long range, int u) {
   const int b = u / sh.H, h = u % sh.H, G = sh.G;
   const long long f = pre[u] / range, l = (pre[u + 1] - 1) / range;
   const int n = (int)(l - f + 1);
   const int seg_f = u - upper_unit(pre, ap.U, f * range);
-  float *Ms = scratch, *Ls = scratch + 16, *fac = scratch + 32;  // fac: [256][G]
-  auto part_of = [&](int i, int g) -> const float * {
-    return partial_ptr(ap, sh, f + i, i == 0 ? seg_f : 0, g);
-  };
-  for (int g = warp; g < G; g += nw) {
-    float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(part_of(i, g)));
-    M = warp_max(M);
-    if (lane == 0) {
-      Ms[g] = M;
-      Ls[g] = 0.f;
-    }
-  }
-  __syncthreads();
-  constexpr int C4 = D / 4;
-  constexpr int OUT_PER_THREAD = 16 * C4 / 128;  // G <= 16 queries, 128 threads
-  float4 acc[OUT_PER_THREAD];
-#pragma unroll
-  for (int r = 0; r < OUT_PER_THREAD; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i0 = 0; i0 < n; i0 += 256) {
-    const int ni = min(256, n - i0);
-    for (int k = tid; k < ni * G; k += blockDim.x) {
-      const int i = i0 + k / G, g = k % G;
-      const float m = __ldcg(part_of(i, g));
-      fac[k] = (m == -INFINITY || Ms[g] == -INFINITY) ? 0.f : exp2f(m - Ms[g]);
-    }
-    __syncthreads();
-    for (int g = warp; g < G; g += nw) {  // fixed summation order: reproducible
-      float ls = 0.f;
-      for (int i = lane; i < ni; i += 32) {
-        const float fv = fac[i * G + g];
-        if (fv != 0.f) ls = fmaf(__ldcg(part_of(i0 + i, g) + 1), fv, ls);
-      }
-      ls = warp_sum(ls);
-      if (lane == 0) Ls[g] += ls;
-    }
-#pragma unroll
-    for (int r = 0; r < OUT_PER_THREAD; ++r) {  // outputs idx = tid + r * blockDim
-      const int idx = tid + r * (int)blockDim.x;
-      if (idx >= G * C4) continue;
-      const int g = idx / C4, c4 = idx % C4;
-      float4 a = acc[r];
-#pragma unroll 8
-      for (int i = 0; i < ni; ++i) {
-        const float fv = fac[i * G + g];
-        const float4 ov = __ldcg(reinterpret_cast<const float4 *>(part_of(i0 + i, g) + kPartO) + c4);
-        a.x = fmaf(ov.x, fv, a.x);
-        a.y = fmaf(ov.y, fv, a.y);
-        a.z = fmaf(ov.z, fv, a.z);
-        a.w = fmaf(ov.w, fv, a.w);
-      }
-      acc[r] = a;
-    }
-    __syncthreads();
-  }
+  constexpr int C4 = D / 4, KB = 8;
   float *o = ap.out + ((size_t)b * sh.Hq + (size_t)h * G) * D;
-#pragma unroll
-  for (int r = 0; r < OUT_PER_THREAD; ++r) {
-    const int idx = tid + r * (int)blockDim.x;
-    if (idx >= G * C4) continue;
+  for (int idx = threadIdx.x; idx < G * C4; idx += blockDim.x) {
     const int g = idx / C4, c4 = idx % C4;
-    const float Lsum = Ls[g];
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    float4 a = acc[r];
+    float M = -INFINITY, Ls = 0.f;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i0 = 0; i0 < n; i0 += KB) {
+      float mm[KB], ll[KB];
+      float4 ov[KB];
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        mm[k] = -INFINITY;
+        ll[k] = 0.f;
+        ov[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i0 + k < n) {
+          const float *pp = partial_ptr(ap, sh, f + i0 + k, i0 + k == 0 ? seg_f : 0, g);
+          mm[k] = __ldcg(pp);
+          ll[k] = __ldcg(pp + 1);
+          ov[k] = __ldcg(reinterpret_cast<const float4 *>(pp + kPartO) + c4);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < KB; ++k) {
+        if (mm[k] == -INFINITY) continue;  // empty partial
+        if (mm[k] > M) {                   // rescale what is accumulated (0 while empty)
+          const float sc = exp2f(M - mm[k]);
+          a.x *= sc;
+          a.y *= sc;
+          a.z *= sc;
+          a.w *= sc;
+          Ls *= sc;
+          M = mm[k];
+        }
+        const float fv = exp2f(mm[k] - M);
+        a.x = fmaf(ov[k].x, fv, a.x);
+        a.y = fmaf(ov[k].y, fv, a.y);
+        a.z = fmaf(ov[k].z, fv, a.z);
+        a.w = fmaf(ov[k].w, fv, a.w);
+        Ls = fmaf(ll[k], fv, Ls);
+      }
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
     a.x *= inv;
     a.y *= inv;
     a.z *= inv;
     a.w *= inv;
     reinterpret_cast<float4 *>(o + (size_t)g * D)[c4] = a;
   }
-  __syncthreads();
+}
+
+// Partial of a segment without rows (the CTA's range only touches the unit's segment
+// overhead): m = -inf marks it empty for combine_unit.
+__device__ __forceinline__ void empty_partial(const Shape &sh, const AttendParams &ap, int seg) {
+  for (int g = threadIdx.x; g < sh.G; g += blockDim.x) {
+    float *pq = partial_ptr(ap, sh, blockIdx.x, seg, g);
+    pq[0] = -INFINITY;
+    pq[1] = 0.f;
+  }
 }
 
 // Counts a finished segment of unit u; true in the thread-block that finished last.
@@ -383,7 +377,7 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
     }
     const int b = u / sh.H, h = u % sh.H;
     const UnitView v = unit_view(sh, c, ap, u);
-    const int wgt = v.gather ? 2 : 1;
+    const int wgt = v.gather ? kCostGather : kCostRow;
     const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, wgt);
     const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, wgt);
     const int ntiles = (r1 - r0 + kAttRows - 1) / kAttRows;
@@ -497,7 +491,7 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
       for (int i = 0; i < D / 32; ++i) sl[2 + lane + 32 * i] = o[g][i];
     }
     merge_warps<D>(sh, ap, scratch, seg);
-    if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u, scratch);
+    if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u);
     start = pre[u + 1];
     ++u;
   }

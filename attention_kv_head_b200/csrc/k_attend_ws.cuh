@@ -207,9 +207,16 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
       break;
     }
     const UnitView v = unit_view(sh, c, ap, u);
-    const int wgt = v.gather ? 2 : 1;
+    const int wgt = v.gather ? kCostGather : kCostRow;
     const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, wgt);
     const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, wgt);
+    if (r1 <= r0) {  // the range only touches this unit's segment overhead
+      empty_partial(sh, ap, seg);
+      if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u);
+      start = pre[u + 1];
+      ++u;
+      continue;
+    }
     const int ntiles = (r1 - r0 + kAttRows - 1) / kAttRows;
     const uint8_t *kring = static_cast<const uint8_t *>(c.k_ring) + (size_t)u * sh.R * rb;
     const uint8_t *vring = static_cast<const uint8_t *>(c.v_ring) + (size_t)u * sh.R * rb;
@@ -300,7 +307,7 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
     __syncthreads();  // every warp is done with its stages: reuse them as scratch
     ws_stage_state<D, NT>(st, sh, scratch, w, lane);
     merge_warps<D>(sh, ap, scratch, seg);
-    if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u, scratch);
+    if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u);
     __syncthreads();  // scratch free before the next segment's copies land
     start = pre[u + 1];
     ++u;

@@ -65,11 +65,19 @@ __device__ __forceinline__ unsigned long long mass_fx(float s, float M, float ta
 
 constexpr int kBins = 2048;            // first-level bins over the distance below the max
 constexpr float kBinsPerUnit = 64.f;   // bin width: 1/64 of a score unit
-constexpr int kCandMax = 4096;         // threshold-bin candidates kept in shared memory
+constexpr int kCandMax = 3072;         // threshold-bin candidates kept in shared memory
+constexpr int kRankMax = 1024;         // candidates resolved by direct ranking
+constexpr int kPartBits = 14;          // per-bin mass held as three 32-bit partial sums
+constexpr uint32_t kPartMask = (1u << kPartBits) - 1u;
+constexpr int kMaxSelectRows = 1 << 18;  // 2^14 x 2^18 fits a 32-bit partial sum
 
-// Dynamic shared memory of topp_kernel: histograms, candidate keys, score cache.
+// Dynamic shared memory of topp_kernel:
+//   [0, 16K)   hmass u64[kBins]   (rank path: sorted mass u64[1024], key u32[1024], pos[1024])
+//   [16K, 24K) hcnt  u32[kBins]
+//   [24K, 48K) hpart u32[3][kBins] (after level 1: candidate keys and positions)
+//   [48K, ...) score cache f32[cache_n]
 __host__ __device__ inline size_t topp_smem_bytes(int cache_n) {
-  return (size_t)kBins * 8 + (size_t)kBins * 4 + (size_t)kCandMax * 4 + (size_t)cache_n * 4;
+  return (size_t)kBins * 8 + (size_t)kBins * 4 + (size_t)3 * kBins * 4 + (size_t)cache_n * 4;
 }
 
 struct SelShared {
@@ -81,6 +89,10 @@ struct SelShared {
   uint32_t sel_cnt;
   unsigned long long sel_mass;
   int ncand;
+  uint32_t theta;  // key of the last kept candidate
+  int pos_cut;     // its local position: equal keys at positions <= pos_cut are kept
+  int n_keep;
+  int clamped;
 };
 
 // Finds, over bins visited in order k = 0..nb-1 (bin(k) = lo_first ? k : nb-1-k), the
@@ -167,9 +179,14 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
 // index list sp_idx / n_kept (positions of kept candidates in ascending order).
 //
 // Level 1: 2048 bins by distance below the max score (width 1/64 score unit; the last
-// bin holds everything further down), exact fixed-point mass and count per bin; the
-// bin where the kept prefix ends is found by a scan. Level 2: a radix select (11 + 11
-// + 10 bits of the order-preserving key) over that bin's elements only.
+// bin holds everything further down) with exact fixed-point mass and count per bin
+// (three 14-bit partial sums per bin so every shared-memory update is a native 32-bit
+// reduction); a scan picks the bin b1 where the kept prefix ends. Level 2 resolves the
+// last kept candidate inside b1: up to kRankMax candidates are ranked directly by
+// (key desc, position asc) and cut by a prefix sum of their masses; larger bins fall
+// back to a radix select (11 + 11 + 10 key bits). The result is the pair
+// (theta, pos_cut): candidate j is kept iff key_j > theta, or key_j == theta and
+// j <= pos_cut.
 template <bool WRITE_IDX>
 __global__ void __launch_bounds__(kSelThreads)
     topp_kernel(Shape sh, Cache c, const float *__restrict__ scores,
@@ -180,74 +197,83 @@ __global__ void __launch_bounds__(kSelThreads)
   pdl_launch();
   if (!unit_active(select_mode, c.moved, b)) return;
   __shared__ SelShared S;
-  extern __shared__ unsigned long long sel_dyn[];
+  __shared__ __align__(8) uint64_t fill_bar;
+  extern __shared__ __align__(16) unsigned long long sel_dyn[];
   unsigned long long *hmass = sel_dyn;                                   // [kBins]
   uint32_t *hcnt = reinterpret_cast<uint32_t *>(hmass + kBins);          // [kBins]
-  uint32_t *ckey = hcnt + kBins;                                         // [kCandMax]
-  float *score_cache = reinterpret_cast<float *>(ckey + kCandMax);      // [cache_n]
+  uint32_t *hpart = hcnt + kBins;                                        // [3][kBins]
+  uint32_t *ckey = hpart;                                                // [kCandMax]
+  int *cpos = reinterpret_cast<int *>(hpart + kCandMax);                 // [kCandMax]
+  float *score_cache = reinterpret_cast<float *>(hpart + 3 * kBins);     // [cache_n]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t lt_mask = (1u << lane) - 1u;
   const Bounds bd = load_bounds(c, b, sh.R);
   if (!bd.ok && tid == 0) flag(c.status, HARDKV_DEV_BAD_BOUNDS);
   const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
   const float *sc = scores + (size_t)u * sh.R;
   const float tv = tau ? tau[u] : 1.0f;
+  const bool cached = L <= cache_n;
+  const float *src = cached ? score_cache : sc;
 
-  // max score from the per-tile partial maxima
+  // scores -> shared memory by one bulk copy (overlaps the max reduction); the row
+  // start is 256-byte aligned (R is a multiple of 64) and ceil4(L) <= R
+  const uint32_t fill_bytes = (uint32_t)((L + 3) & ~3) * 4u;
+  if (cached && L > 0 && tid == 0) {
+    mbar_init(&fill_bar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&fill_bar, fill_bytes);
+    bulk_g2s(score_cache, sc, fill_bytes, &fill_bar);
+  }
+  for (int i = tid; i < kBins; i += kSelThreads) {
+    hcnt[i] = 0;
+    hpart[i] = 0;
+    hpart[kBins + i] = 0;
+    hpart[2 * kBins + i] = 0;
+  }
+  if (tid == 0) {
+    S.ncand = 0;
+    S.n_keep = -1;
+  }
+  // max score from the per-tile partial maxima (block_max synchronises)
   const TileSpan ts = tile_span(bd);
   float m = -INFINITY;
   for (int i = tid; i < ts.n * kPartsPerTile; i += kSelThreads)
     m = fmaxf(m, tile_max[(size_t)u * tm_stride + i]);
-  const float M = block_max(m, S.red);
-  const float *src = sc;
-  if (L <= cache_n) {  // one coalesced sweep from L2, then every sweep reads shared memory
-#pragma unroll 8
-    for (int j = tid; j < L; j += kSelThreads) score_cache[j] = sc[j];
-    src = score_cache;
-  }
-  for (int i = tid; i < kBins; i += kSelThreads) {
-    hcnt[i] = 0;
-    hmass[i] = 0;
-  }
-  if (tid == 0) S.ncand = 0;
-  __syncthreads();
+  const float M = block_max(m, S.red);  // also publishes fill_bar's initialisation
+  if (cached && L > 0 && !mbar_wait(&fill_bar, 0) && tid == 0)
+    flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
 
   const uint32_t cap = (uint32_t)sh.cap;
   auto bin_of = [&](float s) { return min(kBins - 1, (int)((M - s) * kBinsPerUnit)); };
-  // level 1 histogram
-  constexpr int kBatch = 4;
-  for (int base = 0; base < L; base += kBatch * kSelThreads) {
-    float sv[kBatch];
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int j = base + k * kSelThreads + tid;
-      sv[k] = j < L ? src[j] : 0.f;
-    }
-#pragma unroll
-    for (int k = 0; k < kBatch; ++k) {
-      const int j = base + k * kSelThreads + tid;
-      if (j < L) {
-        const int bin = bin_of(sv[k]);
-        atomicAdd(&hcnt[bin], 1u);
-        atomicAdd(&hmass[bin], mass_fx(sv[k], M, tv));
-      }
-    }
+  // level 1: per-bin count and mass; the thread's own mass total for Z
+  unsigned long long zt = 0;
+#pragma unroll 4
+  for (int j = tid; j < L; j += kSelThreads) {
+    const float s = src[j];
+    const int bin = bin_of(s);
+    const unsigned long long mf = mass_fx(s, M, tv);
+    zt += mf;
+    atomicAdd(&hcnt[bin], 1u);
+    atomicAdd(&hpart[bin], (uint32_t)mf & kPartMask);
+    atomicAdd(&hpart[kBins + bin], (uint32_t)(mf >> kPartBits) & kPartMask);
+    atomicAdd(&hpart[2 * kBins + bin], (uint32_t)(mf >> (2 * kPartBits)));
   }
-  __syncthreads();
-  // total mass Z and the threshold T = ceil(p Z) (p >= 1 keeps all)
-  unsigned long long zl = 0;
-  for (int i = tid; i < kBins; i += kSelThreads) zl += hmass[i];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) zl += __shfl_xor_sync(0xffffffffu, zl, o);
-  if (lane == 0) S.wmass[warp] = zl;
+  for (int o = 16; o > 0; o >>= 1) zt += __shfl_xor_sync(0xffffffffu, zt, o);
+  if (lane == 0) S.wmass[warp] = zt;
   __syncthreads();
+  for (int i = tid; i < kBins; i += kSelThreads)
+    hmass[i] = (unsigned long long)hpart[i] +
+               ((unsigned long long)hpart[kBins + i] << kPartBits) +
+               ((unsigned long long)hpart[2 * kBins + i] << (2 * kPartBits));
   unsigned long long Z = 0;
   for (int w = 0; w < kSelThreads / 32; ++w) Z += S.wmass[w];
   __syncthreads();
+  // the threshold T = ceil(p Z) (p >= 1 keeps all)
   const unsigned long long T = p >= 1.0f ? ~0ull : (unsigned long long)ceil((double)p * (double)Z);
 
-  uint32_t above_cnt = 0, E = 0;
-  unsigned long long above_mass = 0, mth = 0;
-  uint32_t theta = 0;
+  uint32_t above_cnt = 0;
+  unsigned long long above_mass = 0;
   bool keep_all = (L == 0);
   int b1 = -1;
   if (!keep_all) {
@@ -255,151 +281,194 @@ __global__ void __launch_bounds__(kSelThreads)
     keep_all = b1 < 0;
   }
   if (!keep_all) {
-    // candidates: the elements of bin b1 (every element with a key equal to theta is one)
-    for (int j = tid; j < L; j += kSelThreads) {
-      const float s = src[j];
-      if (bin_of(s) == b1) {
-        const int k = atomicAdd(&S.ncand, 1);
-        if (k < kCandMax) ckey[k] = order_key(s);
+    // candidates: the elements of bin b1 (every element with the threshold key is one)
+    for (int j0 = 0; j0 < L; j0 += kSelThreads) {
+      const int j = j0 + tid;
+      const float s = j < L ? src[j] : 0.f;
+      const bool member = j < L && bin_of(s) == b1;
+      const unsigned bal = __ballot_sync(0xffffffffu, member);
+      if (bal) {
+        int base = 0;
+        if (lane == 0) base = atomicAdd(&S.ncand, __popc(bal));
+        base = __shfl_sync(0xffffffffu, base, 0);
+        const int k = base + __popc(bal & lt_mask);
+        if (member && k < kCandMax) {
+          ckey[k] = order_key(s);
+          cpos[k] = j;
+        }
       }
     }
     __syncthreads();
     const int ncand = S.ncand;
-    const bool in_list = ncand <= kCandMax;
-    uint32_t prefix = 0, pmask = 0;
-    for (int pass = 0; pass < 3; ++pass) {
-      const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-      const int nb = pass == 2 ? 1024 : 2048;
-      for (int i = tid; i < nb; i += kSelThreads) {
-        hcnt[i] = 0;
-        hmass[i] = 0;
-      }
-      __syncthreads();
-      const int n_it = in_list ? ncand : L;
-      for (int i = tid; i < n_it; i += kSelThreads) {
-        uint32_t key;
-        bool member = true;
-        if (in_list) {
-          key = ckey[i];
-        } else {
-          const float s = src[i];
-          member = bin_of(s) == b1;
-          key = order_key(s);
-        }
-        if (member && (key & pmask) == prefix) {
-          const uint32_t bin = (key >> shift) & (uint32_t)(nb - 1);
-          atomicAdd(&hcnt[bin], 1u);
-          atomicAdd(&hmass[bin], mass_fx(key_to_float(key), M, tv));
+    if (ncand <= kRankMax) {
+      // rank every candidate by (key desc, position asc): gpc threads per candidate
+      unsigned long long *smass = hmass;                                    // [kRankMax]
+      uint32_t *skey = reinterpret_cast<uint32_t *>(hmass + kRankMax);      // [kRankMax]
+      int *spos = reinterpret_cast<int *>(skey + kRankMax);                 // [kRankMax]
+      int gpc = 32;
+      while (gpc > 1 && ncand * gpc > kSelThreads) gpc >>= 1;
+      const int i = tid / gpc, sub = tid % gpc;
+      int rank = 0;
+      uint32_t ki = 0;
+      int pi = 0;
+      if (i < ncand) {
+        ki = ckey[i];
+        pi = cpos[i];
+        for (int jj = sub; jj < ncand; jj += gpc) {
+          const uint32_t kj = ckey[jj];
+          rank += (kj > ki) || (kj == ki && cpos[jj] < pi);
         }
       }
-      __syncthreads();
-      const int sb = select_bin(S, hcnt, hmass, nb, false, above_cnt, above_mass, T, cap);
-      if (sb < 0) {  // cannot happen: bin b1 reaches the threshold; keep everything above
-        keep_all = true;
-        break;
-      }
-      prefix |= (uint32_t)sb << shift;
-      pmask |= (uint32_t)(nb - 1) << shift;
-      if (pass == 2) {
-        E = hcnt[sb];
-        mth = E ? hmass[sb] / E : 0;
+      for (int o = gpc >> 1; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+      if (i < ncand && sub == 0) {
+        skey[rank] = ki;
+        spos[rank] = pi;
+        smass[rank] = mass_fx(key_to_float(ki), M, tv);
       }
       __syncthreads();
-    }
-    theta = prefix;
-  }
-
-  // candidates with key == theta to keep (lowest positions first)
-  uint32_t r = 0, n = (uint32_t)L;
-  bool clamped = false;
-  if (!keep_all) {
-    const unsigned long long need = T > above_mass ? T - above_mass : 0ull;
-    uint32_t r_mass = E;
-    if (T != ~0ull && mth > 0) {
-      const unsigned long long qq = (need + mth - 1) / mth;
-      r_mass = qq < E ? (uint32_t)qq : E;
-    }
-    const uint32_t r_cap = cap - above_cnt;
-    r = min(E, min(r_mass, r_cap));
-    n = above_cnt + r;
-    clamped = (n == cap) && (above_mass + (unsigned long long)r * mth < T);
-  }
-  const bool need_rank = !keep_all && r < E;
-  int32_t *idx = WRITE_IDX ? c.sp_idx + (size_t)u * sh.cap : nullptr;
-  auto kept_at = [&](int j, int rank_ok) -> bool {
-    if (j >= L) return false;
-    if (keep_all) return true;
-    const uint32_t key = order_key(src[j]);
-    return key > theta || (key == theta && rank_ok);
-  };
-  const int nchunks = (L + kSelThreads - 1) / kSelThreads;
-  if (!need_rank && nchunks <= kBins / 32) {
-    // mask words per warp and chunk; then one scan over the words for the slots
-    int *wc = reinterpret_cast<int *>(hcnt);  // [nchunks * 32] words' kept counts
-    for (int ch = 0; ch < nchunks; ++ch) {
-      const int j = ch * kSelThreads + tid;
-      const unsigned word = __ballot_sync(0xffffffffu, kept_at(j, 1));
-      if (lane == 0) {
-        if (mask) mask[(size_t)u * sh.mask_words + ch * 32 + warp] = word;
-        wc[ch * 32 + warp] = __popc(word);
-      }
-    }
-    if (WRITE_IDX) {
-      __syncthreads();
-      // exclusive scan of wc[0 .. nchunks*32) (two entries per thread)
-      const int nw = nchunks * 32;
-      const int a0 = 2 * tid < nw ? wc[2 * tid] : 0, a1 = 2 * tid + 1 < nw ? wc[2 * tid + 1] : 0;
-      int incl = a0 + a1;
+      // prefix mass over the sorted candidates; the cut is where (T, cap) is first reached
+      const unsigned long long mv = tid < ncand ? smass[tid] : 0ull;
+      unsigned long long incl = mv;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (lane == 31) S.scan[warp] = incl;
+      if (lane == 31) S.wmass[warp] = incl;
       __syncthreads();
-      int before = 0;
-      for (int w = 0; w < warp; ++w) before += S.scan[w];
-      const int ex = before + incl - (a0 + a1);
+      for (int w = 0; w < warp; ++w) incl += S.wmass[w];
+      if (tid < ncand) {
+        const unsigned long long m_in = above_mass + incl, m_ex = m_in - mv;
+        const uint32_t c_in = above_cnt + (uint32_t)tid + 1u, c_ex = c_in - 1u;
+        if ((m_in >= T || c_in >= cap) && !(m_ex >= T || c_ex >= cap)) {
+          S.theta = skey[tid];
+          S.pos_cut = spos[tid];
+          S.n_keep = (int)c_in;
+          S.clamped = (c_in == cap) && (m_in < T);
+        }
+      }
       __syncthreads();
-      if (2 * tid < nw) wc[2 * tid] = ex;
-      if (2 * tid + 1 < nw) wc[2 * tid + 1] = ex + a0;
-      __syncthreads();
-      for (int ch = 0; ch < nchunks; ++ch) {
-        const int j = ch * kSelThreads + tid;
-        const bool kept = kept_at(j, 1);
-        const unsigned word = __ballot_sync(0xffffffffu, kept);
-        const int slot = wc[ch * 32 + warp] + __popc(word & ((1u << lane) - 1u));
-        if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
+    } else {
+      // radix select over bin b1 (11 + 11 + 10 key bits), the list in shared memory
+      // when it fits, else a rescan of the unit's scores
+      const bool in_list = ncand <= kCandMax;
+      uint32_t prefix = 0, pmask = 0, E = 0;
+      unsigned long long mth = 0;
+      bool found = true;
+      for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const int nb = pass == 2 ? 1024 : 2048;
+        for (int q = tid; q < nb; q += kSelThreads) {
+          hcnt[q] = 0;
+          hmass[q] = 0;
+        }
+        __syncthreads();
+        const int n_it = in_list ? ncand : L;
+        for (int q = tid; q < n_it; q += kSelThreads) {
+          uint32_t key;
+          bool member = true;
+          if (in_list) {
+            key = ckey[q];
+          } else {
+            const float s = src[q];
+            member = bin_of(s) == b1;
+            key = order_key(s);
+          }
+          if (member && (key & pmask) == prefix) {
+            const uint32_t bin = (key >> shift) & (uint32_t)(nb - 1);
+            atomicAdd(&hcnt[bin], 1u);
+            atomicAdd(&hmass[bin], mass_fx(key_to_float(key), M, tv));
+          }
+        }
+        __syncthreads();
+        const int sb = select_bin(S, hcnt, hmass, nb, false, above_cnt, above_mass, T, cap);
+        if (sb < 0) {  // cannot happen: bin b1 reaches the threshold
+          found = false;
+          break;
+        }
+        prefix |= (uint32_t)sb << shift;
+        pmask |= (uint32_t)(nb - 1) << shift;
+        if (pass == 2) {
+          E = hcnt[sb];
+          mth = E ? hmass[sb] / E : 0;
+        }
+        __syncthreads();
+      }
+      if (found) {
+        // r of the E candidates with key == theta are kept, lowest positions first
+        const unsigned long long need = T > above_mass ? T - above_mass : 0ull;
+        uint32_t r_mass = E;
+        if (T != ~0ull && mth > 0) {
+          const unsigned long long qq = (need + mth - 1) / mth;
+          r_mass = qq < E ? (uint32_t)qq : E;
+        }
+        const uint32_t r = min(E, min(r_mass, cap - above_cnt));
+        // position of the r-th element with key == theta
+        int run_eq = 0;
+        for (int j0 = 0; j0 < L; j0 += kSelThreads) {
+          const int j = j0 + tid;
+          const bool eq = j < L && order_key(src[j]) == prefix;
+          const int2 e = block_scan_flag(eq, S.scan);
+          if (eq && run_eq + e.x == (int)r - 1) S.pos_cut = j;
+          run_eq += e.y;
+        }
+        if (tid == 0) {
+          S.theta = prefix;
+          S.n_keep = (int)(above_cnt + r);
+          S.clamped = (above_cnt + r == cap) && (above_mass + (unsigned long long)r * mth < T);
+        }
+        __syncthreads();
       }
     }
-  } else {
-    int run_eq = 0, run_kept = 0;
-    for (int ch = 0; ch < nchunks; ++ch) {
-      const int j = ch * kSelThreads + tid;
-      const bool eq = j < L && order_key(src[j]) == theta;
-      const int2 e = block_scan_flag(eq, S.scan);
-      const bool kept = kept_at(j, !need_rank || run_eq + e.x < (int)r);
-      run_eq += e.y;
-      const unsigned word = __ballot_sync(0xffffffffu, kept);
-      if (mask && lane == 0) mask[(size_t)u * sh.mask_words + ch * 32 + warp] = word;
-      if (WRITE_IDX) {
-        const int2 k2 = block_scan_flag(kept, S.scan);
-        const int slot = run_kept + k2.x;
-        if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
-        run_kept += k2.y;
-      }
+    if (S.n_keep < 0) {  // no cut found (not reachable): keep everything, flag it
+      keep_all = true;
+      if (tid == 0) flag(c.status, HARDKV_DEV_SELECT);
     }
   }
-  if (mask) {
-    const int w0 = nchunks * 32;
-    for (int w = w0 + tid; w < sh.mask_words; w += kSelThreads) mask[(size_t)u * sh.mask_words + w] = 0u;
+
+  // mask words and compact indices: warp w owns words [w K, (w+1) K), bit = lane
+  const uint32_t theta = keep_all ? 0u : S.theta;
+  const int pos_cut = keep_all ? 0x7fffffff : S.pos_cut;
+  const int n = keep_all ? min(L, sh.cap) : S.n_keep;
+  auto kept_at = [&](int j) -> bool {
+    if (j >= L) return false;
+    const uint32_t key = order_key(src[j]);
+    return key > theta || (key == theta && j <= pos_cut);
+  };
+  const int nwords = (L + 31) >> 5;
+  const int K = (nwords + kSelThreads / 32 - 1) / (kSelThreads / 32);
+  uint32_t *mrow = mask ? mask + (size_t)u * sh.mask_words : nullptr;
+  int wcount = 0;
+  for (int k = 0; k < K; ++k) {
+    const int wi = warp * K + k;
+    if (wi >= nwords) break;
+    const unsigned word = __ballot_sync(0xffffffffu, kept_at(wi * 32 + lane));
+    if (mrow && lane == 0) mrow[wi] = word;
+    wcount += __popc(word);
   }
+  if (mrow)
+    for (int wi = nwords + tid; wi < sh.mask_words; wi += kSelThreads) mrow[wi] = 0u;
   if (WRITE_IDX) {
-    for (int s2 = (int)n + tid; s2 < sh.cap; s2 += kSelThreads) idx[s2] = -1;
-    if (tid == 0) c.n_kept[u] = (int)n;
+    int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
+    if (lane == 0) S.scan[warp] = wcount;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += S.scan[w];
+    for (int k = 0; k < K; ++k) {
+      const int wi = warp * K + k;
+      if (wi >= nwords) break;
+      const int j = wi * 32 + lane;
+      const bool kept = kept_at(j);
+      const unsigned word = __ballot_sync(0xffffffffu, kept);
+      const int slot = base + __popc(word & lt_mask);
+      if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
+      base += __popc(word);
+    }
+    for (int s2 = n + tid; s2 < sh.cap; s2 += kSelThreads) idx[s2] = -1;
+    if (tid == 0) c.n_kept[u] = n;
   }
   if (tid == 0) {
-    if (clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
+    if (!keep_all && S.clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
     atomicAdd(c.status + HARDKV_ST_SELECTIONS, 1u);
   }
 }

@@ -79,6 +79,7 @@ enum {
 #define HARDKV_DEV_BAD_BOUNDS    2u  /* s_lo <= d_lo <= len broken or span > R: unit skipped */
 #define HARDKV_DEV_SEGMENTS      4u  /* attention partition had to drop a segment */
 #define HARDKV_DEV_WAIT_TIMEOUT  8u  /* a pipeline wait hit its iteration limit */
+#define HARDKV_DEV_SELECT       16u  /* top-p found no cut (inconsistent input): unit kept all */
 
 /* Static shape of one attention layer's cascade cache. */
 typedef struct {
@@ -91,8 +92,9 @@ typedef struct {
   int32_t condensed_slots;  /* C: Condensed slots per (b,h), >= 1 (<= 2048 for MERGE) */
   int32_t n_sink;           /* slots [0, n_sink) are pinned (never merged into) */
   int32_t sparse_cap;       /* Cap: compact rows per (b,h), >= 1 */
-  int32_t ring_rows;        /* R: raw rows per (b,h); multiple of 64; the live span
-                               [s_lo, len) must stay <= R (R >= Sparse + W + block) */
+  int32_t ring_rows;        /* R: raw rows per (b,h); multiple of 64, <= 262144; the
+                               live span [s_lo, len) must stay <= R
+                               (R >= Sparse + W + block) */
   int32_t dtype;            /* HARDKV_F32 or HARDKV_BF16 */
   int32_t condense_mode;    /* HARDKV_EVICT or HARDKV_MERGE */
 } hardkv_desc;

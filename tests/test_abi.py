@@ -45,11 +45,16 @@ def test_north_star_entry_points_declared():
     ("n_q_heads", 8 * 17, B.EINVAL), ("head_dim", 96, B.EINVAL), ("block", 0, B.EINVAL),
     ("condensed_slots", 0, B.EINVAL), ("n_sink", 300, B.EINVAL), ("sparse_cap", 0, B.ECAP),
     ("ring_rows", 8001, B.ECAP), ("ring_rows", 192, B.ECAP), ("dense_window", 7990, B.ECAP), ("condense_mode", 3, B.EINVAL),
+    ("ring_rows", (1 << 18) + 64, B.EINVAL),   # per-bin partial mass sums are 32-bit
 ])
 def test_validate_rejects(lib, field, value, code):
     d = desc(**{field: value})
     assert lib.hardkv_validate(ctypes.byref(d)) == code
     assert lib.hardkv_workspace_bytes(ctypes.byref(d)) == 0
+
+
+def test_ring_rows_limit_inclusive(lib):
+    assert lib.hardkv_validate(ctypes.byref(desc(ring_rows=1 << 18))) == B.OK
 
 
 def test_validate_accepts_all_workloads(lib):
