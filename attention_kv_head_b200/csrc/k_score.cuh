@@ -15,6 +15,7 @@ namespace hardkv {
 
 constexpr int kTile = 64;         // key rows per tile (ring rows are 64-aligned)
 constexpr int kPartsPerTile = 4;  // per-warp partial maxima per tile
+constexpr int kScoreChunk = 2;    // consecutive tiles a CTA takes before the next CTA
 
 template <int D>
 struct ScoreTma {
@@ -123,17 +124,22 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
   }
   __syncthreads();
 
+  // tile order: chunks of kScoreChunk consecutive tiles dealt round-robin to the CTAs,
+  // so the CTAs sweep the keys together (neighbouring rows in flight at any time)
   const long long total = pre[sh.B];
-  const long long g0 = total * blockIdx.x / gridDim.x;
-  const long long g1 = total * (blockIdx.x + 1) / gridDim.x;
-  if (g0 >= g1) return;
+  const long long nchunks = (total + kScoreChunk - 1) / kScoreChunk;
+  if ((long long)blockIdx.x >= nchunks) return;
+  auto tile_of = [&](long long i) -> long long {  // this CTA's i-th tile; >= total: done
+    const long long ch = (long long)blockIdx.x + (i / kScoreChunk) * gridDim.x;
+    return ch * kScoreChunk + i % kScoreChunk;
+  };
 
   if (warp == Cfg::CONSUMER_WARPS) {
     // ---------------- producer: one thread issues the TMA loads
     if (lane != 0) return;
     int b = 0;
     long long issued = 0;
-    for (long long g = g0; g < g1; ++g, ++issued) {
+    for (long long g = tile_of(0); g < total; g = tile_of(++issued)) {
       while (g >= pre[b + 1]) ++b;
       const int idx = (int)(g - pre[b]);
       const int h = idx / ntile[b], lt = idx % ntile[b];
@@ -165,7 +171,7 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
   uint32_t qb[NT][D / 16][2];
   int cur_u = -1, b = 0;
   long long i = 0;
-  for (long long gg = g0; gg < g1; ++gg, ++i) {
+  for (long long gg = tile_of(0); gg < total; gg = tile_of(++i)) {
     while (gg >= pre[b + 1]) ++b;
     const int idx = (int)(gg - pre[b]);
     if ((int)(i & 1) != group) continue;

@@ -171,6 +171,21 @@ __device__ __forceinline__ int select_bin(SelShared &S, const uint32_t *cnt,
   return sb;
 }
 
+// Exclusive prefix at index `warp` of 32 per-warp values in shared memory, by one
+// shuffle scan (every lane of the calling warp gets it).
+static_assert(kSelThreads == 1024, "one value per lane: 32 warps");
+template <typename V>
+__device__ __forceinline__ V warp_prefix_of(const V *v, int warp, int lane) {
+  const V x = v[lane];
+  V incl = x;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const V y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  return __shfl_sync(0xffffffffu, incl - x, warp);
+}
+
 __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
@@ -244,48 +259,60 @@ __global__ void __launch_bounds__(kSelThreads)
     flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
 
   const uint32_t cap = (uint32_t)sh.cap;
-  auto bin_of = [&](float s) { return min(kBins - 1, (int)((M - s) * kBinsPerUnit)); };
-  // level 1: per-bin count and mass; the thread's own mass total for Z
-  unsigned long long zt = 0;
+  // p >= 1 with at most Cap candidates keeps every candidate: no histogram needed
+  bool keep_all = L == 0 || (p >= 1.0f && (uint32_t)L <= cap);
+  // per-bin counts matter only when Cap can bind before the last candidate; otherwise
+  // the count above b1 comes from the candidate pass
+  const bool use_cnt = cap < (uint32_t)L;
+  // clamped both ways: a NaN or inf score must not index outside the bins
+  auto bin_of = [&](float s) { return max(0, min(kBins - 1, (int)((M - s) * kBinsPerUnit))); };
+  unsigned long long T = ~0ull;
+  if (!keep_all) {
+    // level 1: per-bin count and mass; the thread's own mass total for Z
+    unsigned long long zt = 0;
 #pragma unroll 4
-  for (int j = tid; j < L; j += kSelThreads) {
-    const float s = src[j];
-    const int bin = bin_of(s);
-    const unsigned long long mf = mass_fx(s, M, tv);
-    zt += mf;
-    atomicAdd(&hcnt[bin], 1u);
-    atomicAdd(&hpart[bin], (uint32_t)mf & kPartMask);
-    atomicAdd(&hpart[kBins + bin], (uint32_t)(mf >> kPartBits) & kPartMask);
-    atomicAdd(&hpart[2 * kBins + bin], (uint32_t)(mf >> (2 * kPartBits)));
-  }
+    for (int j = tid; j < L; j += kSelThreads) {
+      const float s = src[j];
+      const int bin = bin_of(s);
+      const unsigned long long mf = mass_fx(s, M, tv);
+      zt += mf;
+      if (use_cnt) atomicAdd(&hcnt[bin], 1u);
+      atomicAdd(&hpart[bin], (uint32_t)mf & kPartMask);
+      atomicAdd(&hpart[kBins + bin], (uint32_t)(mf >> kPartBits) & kPartMask);
+      atomicAdd(&hpart[2 * kBins + bin], (uint32_t)(mf >> (2 * kPartBits)));
+    }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) zt += __shfl_xor_sync(0xffffffffu, zt, o);
-  if (lane == 0) S.wmass[warp] = zt;
-  __syncthreads();
-  for (int i = tid; i < kBins; i += kSelThreads)
-    hmass[i] = (unsigned long long)hpart[i] +
-               ((unsigned long long)hpart[kBins + i] << kPartBits) +
-               ((unsigned long long)hpart[2 * kBins + i] << (2 * kPartBits));
-  unsigned long long Z = 0;
-  for (int w = 0; w < kSelThreads / 32; ++w) Z += S.wmass[w];
-  __syncthreads();
-  // the threshold T = ceil(p Z) (p >= 1 keeps all)
-  const unsigned long long T = p >= 1.0f ? ~0ull : (unsigned long long)ceil((double)p * (double)Z);
+    for (int o = 16; o > 0; o >>= 1) zt += __shfl_xor_sync(0xffffffffu, zt, o);
+    if (lane == 0) S.wmass[warp] = zt;
+    __syncthreads();
+    for (int i = tid; i < kBins; i += kSelThreads)
+      hmass[i] = (unsigned long long)hpart[i] +
+                 ((unsigned long long)hpart[kBins + i] << kPartBits) +
+                 ((unsigned long long)hpart[2 * kBins + i] << (2 * kPartBits));
+    unsigned long long Z = 0;
+    for (int w = 0; w < kSelThreads / 32; ++w) Z += S.wmass[w];
+    __syncthreads();
+    // the threshold T = ceil(p Z) (p >= 1 keeps all, up to Cap)
+    if (p < 1.0f) T = (unsigned long long)ceil((double)p * (double)Z);
+  }
 
   uint32_t above_cnt = 0;
   unsigned long long above_mass = 0;
-  bool keep_all = (L == 0);
   int b1 = -1;
   if (!keep_all) {
     b1 = select_bin(S, hcnt, hmass, kBins, true, above_cnt, above_mass, T, cap);
     keep_all = b1 < 0;
   }
   if (!keep_all) {
-    // candidates: the elements of bin b1 (every element with the threshold key is one)
+    // candidates: the elements of bin b1 (every element with the threshold key is one);
+    // without per-bin counts, also the number of elements above b1
+    uint32_t n_above = 0;
     for (int j0 = 0; j0 < L; j0 += kSelThreads) {
       const int j = j0 + tid;
       const float s = j < L ? src[j] : 0.f;
-      const bool member = j < L && bin_of(s) == b1;
+      const int bn = j < L ? bin_of(s) : kBins;
+      const bool member = bn == b1;
+      if (!use_cnt) n_above += __popc(__ballot_sync(0xffffffffu, bn < b1));
       const unsigned bal = __ballot_sync(0xffffffffu, member);
       if (bal) {
         int base = 0;
@@ -298,8 +325,13 @@ __global__ void __launch_bounds__(kSelThreads)
         }
       }
     }
+    if (!use_cnt && lane == 0) S.scan[warp] = (int)n_above;
     __syncthreads();
     const int ncand = S.ncand;
+    if (!use_cnt) {
+      above_cnt = 0;
+      for (int w = 0; w < kSelThreads / 32; ++w) above_cnt += (uint32_t)S.scan[w];
+    }
     if (ncand <= kRankMax) {
       // rank every candidate by (key desc, position asc): gpc threads per candidate
       unsigned long long *smass = hmass;                                    // [kRankMax]
@@ -336,7 +368,7 @@ __global__ void __launch_bounds__(kSelThreads)
       }
       if (lane == 31) S.wmass[warp] = incl;
       __syncthreads();
-      for (int w = 0; w < warp; ++w) incl += S.wmass[w];
+      incl += warp_prefix_of(S.wmass, warp, lane);
       if (tid < ncand) {
         const unsigned long long m_in = above_mass + incl, m_ex = m_in - mv;
         const uint32_t c_in = above_cnt + (uint32_t)tid + 1u, c_ex = c_in - 1u;
@@ -344,7 +376,7 @@ __global__ void __launch_bounds__(kSelThreads)
           S.theta = skey[tid];
           S.pos_cut = spos[tid];
           S.n_keep = (int)c_in;
-          S.clamped = (c_in == cap) && (m_in < T);
+          S.clamped = (c_in == cap) && (T == ~0ull ? (uint32_t)L > cap : m_in < T);
         }
       }
       __syncthreads();
@@ -415,7 +447,8 @@ __global__ void __launch_bounds__(kSelThreads)
         if (tid == 0) {
           S.theta = prefix;
           S.n_keep = (int)(above_cnt + r);
-          S.clamped = (above_cnt + r == cap) && (above_mass + (unsigned long long)r * mth < T);
+          S.clamped = (above_cnt + r == cap) &&
+                      (T == ~0ull ? (uint32_t)L > cap : above_mass + (unsigned long long)r * mth < T);
         }
         __syncthreads();
       }
@@ -438,32 +471,64 @@ __global__ void __launch_bounds__(kSelThreads)
   const int nwords = (L + 31) >> 5;
   const int K = (nwords + kSelThreads / 32 - 1) / (kSelThreads / 32);
   uint32_t *mrow = mask ? mask + (size_t)u * sh.mask_words : nullptr;
-  int wcount = 0;
-  for (int k = 0; k < K; ++k) {
-    const int wi = warp * K + k;
-    if (wi >= nwords) break;
-    const unsigned word = __ballot_sync(0xffffffffu, kept_at(wi * 32 + lane));
-    if (mrow && lane == 0) mrow[wi] = word;
-    wcount += __popc(word);
+  int32_t *idx = WRITE_IDX ? c.sp_idx + (size_t)u * sh.cap : nullptr;
+  constexpr int KW = 8;  // words a warp keeps in registers
+  if (K <= KW) {
+    uint32_t wb[KW];
+    int wcount = 0;
+#pragma unroll
+    for (int k = 0; k < KW; ++k) {
+      const int wi = warp * K + k;
+      wb[k] = 0u;
+      if (k < K && wi < nwords) wb[k] = __ballot_sync(0xffffffffu, kept_at(wi * 32 + lane));
+      wcount += __popc(wb[k]);
+    }
+    if (mrow) {  // lane k stores word k: one coalesced store per warp
+      uint32_t mine = 0u;
+#pragma unroll
+      for (int k = 0; k < KW; ++k) mine = lane == k ? wb[k] : mine;
+      if (lane < K && warp * K + lane < nwords) mrow[warp * K + lane] = mine;
+    }
+    if (WRITE_IDX) {
+      if (lane == 0) S.scan[warp] = wcount;
+      __syncthreads();
+      int base = warp_prefix_of(S.scan, warp, lane);
+#pragma unroll
+      for (int k = 0; k < KW; ++k) {
+        const int wi = warp * K + k;
+        const int slot = base + __popc(wb[k] & lt_mask);
+        if (((wb[k] >> lane) & 1u) && slot < sh.cap) idx[slot] = bd.s_lo + wi * 32 + lane;
+        base += __popc(wb[k]);
+      }
+    }
+  } else {
+    int wcount = 0;
+    for (int k = 0; k < K; ++k) {
+      const int wi = warp * K + k;
+      if (wi >= nwords) break;
+      const unsigned word = __ballot_sync(0xffffffffu, kept_at(wi * 32 + lane));
+      if (mrow && lane == 0) mrow[wi] = word;
+      wcount += __popc(word);
+    }
+    if (WRITE_IDX) {
+      if (lane == 0) S.scan[warp] = wcount;
+      __syncthreads();
+      int base = warp_prefix_of(S.scan, warp, lane);
+      for (int k = 0; k < K; ++k) {
+        const int wi = warp * K + k;
+        if (wi >= nwords) break;
+        const int j = wi * 32 + lane;
+        const bool kept = kept_at(j);
+        const unsigned word = __ballot_sync(0xffffffffu, kept);
+        const int slot = base + __popc(word & lt_mask);
+        if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
+        base += __popc(word);
+      }
+    }
   }
   if (mrow)
     for (int wi = nwords + tid; wi < sh.mask_words; wi += kSelThreads) mrow[wi] = 0u;
   if (WRITE_IDX) {
-    int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
-    if (lane == 0) S.scan[warp] = wcount;
-    __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += S.scan[w];
-    for (int k = 0; k < K; ++k) {
-      const int wi = warp * K + k;
-      if (wi >= nwords) break;
-      const int j = wi * 32 + lane;
-      const bool kept = kept_at(j);
-      const unsigned word = __ballot_sync(0xffffffffu, kept);
-      const int slot = base + __popc(word & lt_mask);
-      if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
-      base += __popc(word);
-    }
     for (int s2 = n + tid; s2 < sh.cap; s2 += kSelThreads) idx[s2] = -1;
     if (tid == 0) c.n_kept[u] = n;
   }
