@@ -190,6 +190,48 @@ __device__ __forceinline__ float key_to_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+// (key desc, position asc): the top-p order of candidates.
+__device__ __forceinline__ bool sel_before(uint32_t ka, int pa, uint32_t kb, int pb) {
+  return ka > kb || (ka == kb && pa < pb);
+}
+
+// Sorts up to 64 (key, position) pairs held two per lane (element e = lane + 32 h) into
+// the top-p order with a bitonic network; pads (key 0, position INT_MAX) sort last.
+__device__ __forceinline__ void warp_sort64(uint32_t (&k)[2], int (&p)[2], int lane) {
+#pragma unroll
+  for (int kk = 2; kk <= 64; kk <<= 1) {
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1) {
+      if (j == 32) {  // partners in the same lane
+        const bool asc = (lane & kk) == 0;  // kk == 64 here: the whole set ascending
+        const bool first = sel_before(k[0], p[0], k[1], p[1]);
+        if (first != asc) {
+          const uint32_t tk = k[0];
+          const int tp = p[0];
+          k[0] = k[1];
+          p[0] = p[1];
+          k[1] = tk;
+          p[1] = tp;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = lane + 32 * h;
+          const uint32_t ok = __shfl_xor_sync(0xffffffffu, k[h], j);
+          const int op = __shfl_xor_sync(0xffffffffu, p[h], j);
+          const bool lower = (e & j) == 0, asc = (e & kk) == 0;
+          const bool mine_first = sel_before(k[h], p[h], ok, op);
+          // the lower index keeps the element that comes first (ascending runs)
+          if ((lower == asc) != mine_first) {
+            k[h] = ok;
+            p[h] = op;
+          }
+        }
+      }
+    }
+  }
+}
+
 // One CTA per (b,h). Writes the mask (if not NULL) and, with WRITE_IDX, the compact
 // index list sp_idx / n_kept (positions of kept candidates in ascending order).
 //
@@ -332,7 +374,49 @@ __global__ void __launch_bounds__(kSelThreads)
       above_cnt = 0;
       for (int w = 0; w < kSelThreads / 32; ++w) above_cnt += (uint32_t)S.scan[w];
     }
-    if (ncand <= kRankMax) {
+    if (ncand <= 64) {
+      // small bins: one warp sorts the candidates and finds the cut (no block barrier)
+      if (warp == 0) {
+        uint32_t kq[2];
+        int pq[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = lane + 32 * h;
+          kq[h] = e < ncand ? ckey[e] : 0u;
+          pq[h] = e < ncand ? cpos[e] : 0x7fffffff;
+        }
+        warp_sort64(kq, pq, lane);
+        unsigned long long run_m = above_mass;
+        uint32_t run_c = above_cnt;
+        bool done = false;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int e = lane + 32 * h;
+          const unsigned long long mv = e < ncand ? mass_fx(key_to_float(kq[h]), M, tv) : 0ull;
+          unsigned long long incl = mv;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const unsigned long long m_in = run_m + incl;
+          const uint32_t c_in = run_c + (uint32_t)lane + 1u;
+          const unsigned hit = __ballot_sync(0xffffffffu, e < ncand && (m_in >= T || c_in >= cap));
+          if (!done && hit) {
+            if (lane == __ffs(hit) - 1) {
+              S.theta = kq[h];
+              S.pos_cut = pq[h];
+              S.n_keep = (int)c_in;
+              S.clamped = (c_in == cap) && (T == ~0ull ? (uint32_t)L > cap : m_in < T);
+            }
+            done = true;
+          }
+          run_m += __shfl_sync(0xffffffffu, incl, 31);
+          run_c += 32u;
+        }
+      }
+      __syncthreads();
+    } else if (ncand <= kRankMax) {
       // rank every candidate by (key desc, position asc): gpc threads per candidate
       unsigned long long *smass = hmass;                                    // [kRankMax]
       uint32_t *skey = reinterpret_cast<uint32_t *>(hmass + kRankMax);      // [kRankMax]
