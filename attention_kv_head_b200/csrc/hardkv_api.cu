@@ -548,6 +548,20 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   return record(ev, 5, stream);
 }
 
+// Device address of a host buffer the GPU can reach in place (pinned and mapped, as
+// cudaHostAlloc memory is under unified addressing), 16-byte aligned; NULL otherwise.
+static void *mapped_host(const void *host) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+    cudaGetLastError();  // pageable memory on older runtimes: not mapped
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr ||
+      reinterpret_cast<uintptr_t>(a.devicePointer) % 16 != 0)
+    return nullptr;
+  return a.devicePointer;
+}
+
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
                             const hardkv_step_args *h, void *ws, cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));
@@ -563,19 +577,27 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   dv.v_new = w + L.st_v;
   dv.out = reinterpret_cast<float *>(w + L.st_out);
   dv.tau = h->tau ? reinterpret_cast<const float *>(w + L.st_tau) : nullptr;
+  // q is read by many CTAs and is copied; k_new / v_new (read once, by the append
+  // kernel) and out (written once per unit) are used in place when the GPU can address
+  // them, which saves three copy latencies per step; other host memory is staged
+  void *k_map = mapped_host(h->k_new), *v_map = mapped_host(h->v_new);
+  void *o_map = mapped_host(h->out);
+  if (k_map) dv.k_new = k_map;
+  if (v_map) dv.v_new = v_map;
+  if (o_map) dv.out = static_cast<float *>(o_map);
   cudaError_t r;
   if ((r = cudaMemcpyAsync(w + L.st_q, h->q, nq * e, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
-      (r = cudaMemcpyAsync(w + L.st_k, h->k_new, U * desc->head_dim * e, cudaMemcpyHostToDevice,
-                           stream)) != cudaSuccess ||
-      (r = cudaMemcpyAsync(w + L.st_v, h->v_new, U * desc->head_dim * e, cudaMemcpyHostToDevice,
-                           stream)) != cudaSuccess)
+      (!k_map && (r = cudaMemcpyAsync(w + L.st_k, h->k_new, U * desc->head_dim * e,
+                                      cudaMemcpyHostToDevice, stream)) != cudaSuccess) ||
+      (!v_map && (r = cudaMemcpyAsync(w + L.st_v, h->v_new, U * desc->head_dim * e,
+                                      cudaMemcpyHostToDevice, stream)) != cudaSuccess))
     return cuda_fail(r, "cudaMemcpyAsync H2D");
   if (h->tau && (r = cudaMemcpyAsync(w + L.st_tau, h->tau, U * 4, cudaMemcpyHostToDevice, stream)) !=
                     cudaSuccess)
     return cuda_fail(r, "cudaMemcpyAsync H2D");
   HKV_TRY(hardkv_decode_step(desc, cache, &dv, ws, stream));
-  if ((r = cudaMemcpyAsync(h->out, w + L.st_out, nq * 4, cudaMemcpyDeviceToHost, stream)) !=
-      cudaSuccess)
+  if (!o_map && (r = cudaMemcpyAsync(h->out, w + L.st_out, nq * 4, cudaMemcpyDeviceToHost, stream)) !=
+                    cudaSuccess)
     return cuda_fail(r, "cudaMemcpyAsync D2H");
   return HARDKV_OK;
 }

@@ -209,7 +209,10 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
  * the copies asynchronous): args->q, k_new, v_new and tau (if not NULL) are read from
  * the host, args->out is written to the host; the copies and the step are enqueued
  * on `stream` and the caller synchronises before reading `out`. args->mask, if not
- * NULL, is a device pointer. Staging buffers live in the workspace. */
+ * NULL, is a device pointer. Staging buffers live in the workspace. Pinned, mapped
+ * and 16-byte aligned k_new, v_new and out buffers (cudaHostAlloc memory under
+ * unified addressing) are read / written by the kernels in place instead of copied;
+ * q and tau are always copied. */
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
                             const hardkv_step_args *host_args, void *ws,
                             cudaStream_t stream);

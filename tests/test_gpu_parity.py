@@ -315,15 +315,20 @@ def test_graph_capture_replays_the_step():
         assert torch.equal(out, out_e) and torch.equal(mask, mask_e)
 
 
-def test_host_entry_point_matches_device_step():
+@pytest.mark.parametrize("pinned", [(1, 1, 1, 1), (0, 0, 0, 0), (1, 1, 0, 1), (0, 1, 1, 0)],
+                         ids=["pinned", "pageable", "mixed_kv", "mixed_out"])
+def test_host_entry_point_matches_device_step(pinned):
+    """Host buffers: pinned mapped ones are used in place by the kernels, pageable ones
+    are staged by copies; every combination gives the device step's result."""
     w = synth.small(batch=2)
     st = synth.initial_state(w)
     dc = DecodeCache.from_state(st)
     dc2 = DecodeCache.from_state(st)
     (q, k, v), _ = U.upload_step(dc, w, st, 0)
     _, out = U.run_fused_step(dc, q, k, v, w.p)
-    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
-    oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+    host = [t.cpu() for t in (q, k, v)] + [torch.full(out.shape, float("nan"))]
+    qh, kh, vh, oh = (t.pin_memory() if pn else t for t, pn in zip(host, pinned))
     dc2.step_host(qh, kh, vh, oh, w.p)
     torch.cuda.synchronize()
     assert torch.equal(oh, out.cpu())
+    assert torch.equal(dc2.len, dc.len) and torch.equal(dc2.sp_idx, dc.sp_idx)
