@@ -337,9 +337,13 @@ int launch_condense(const hardkv_desc *d, const Shape &sh, const Cache &c, cudaS
 
 template <int D, int NT>
 int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
-                     float *scores, float *tm, int tm_stride, int select_mode, cudaStream_t st) {
+                     float *scores, float *tm, int tm_stride, int select_mode, cudaStream_t st,
+                     const CUtensorMap *pre) {
   CUtensorMap map;
-  HKV_TRY(make_kmap(&map, d, c.k_ring));
+  if (pre)
+    map = *pre;
+  else
+    HKV_TRY(make_kmap(&map, d, c.k_ring));
   const size_t smem = ScoreTma<D>::smem_bytes(sh.B);
   HKV_TRY(set_smem(score_tma_kernel<D, NT>, smem));
   static int per_sm = 0;
@@ -351,16 +355,18 @@ int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, cons
   return HARDKV_OK;
 }
 
+// `pre`: the key tensor map when the caller encoded it ahead of its first launch (the
+// fused step does, so no host work sits between its kernel launches); NULL: encode here.
 int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, void *ws,
-                 const Layout &L, int select_mode, cudaStream_t st) {
+                 const Layout &L, int select_mode, cudaStream_t st, const CUtensorMap *pre = nullptr) {
   float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + L.scores);
   float *tm = reinterpret_cast<float *>(static_cast<char *>(ws) + L.tile_max);
   if (d->dtype == HARDKV_BF16) {
     if (sh.G <= 8)
-      return sh.d == 128 ? launch_score_tma<128, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
-                         : launch_score_tma<64, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
-    return sh.d == 128 ? launch_score_tma<128, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st)
-                       : launch_score_tma<64, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st);
+      return sh.d == 128 ? launch_score_tma<128, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre)
+                         : launch_score_tma<64, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre);
+    return sh.d == 128 ? launch_score_tma<128, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre)
+                       : launch_score_tma<64, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre);
   }
   const dim3 grid(sh.R / kTile + 2, sh.B * sh.H);
   launch_pdl(score_f32_kernel, grid, dim3(128), (size_t)sh.G * sh.d * 4, st, sh, c,
@@ -534,13 +540,16 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
   const Layout L = layout(desc);
+  CUtensorMap kmap;
+  const bool tma = desc->dtype == HARDKV_BF16;
+  if (tma) HKV_TRY(make_kmap(&kmap, desc, c.k_ring));  // host work before the first launch
   cudaEvent_t *ev = a->stage_events;
   HKV_TRY(record(ev, 0, stream));
   HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, ws, L, stream));  // zeroes counters
   HKV_TRY(record(ev, 1, stream));
   HKV_TRY(launch_condense(desc, sh, c, stream));
   HKV_TRY(record(ev, 2, stream));
-  HKV_TRY(launch_score(desc, sh, c, a->q, ws, L, a->select_mode, stream));
+  HKV_TRY(launch_score(desc, sh, c, a->q, ws, L, a->select_mode, stream, tma ? &kmap : nullptr));
   HKV_TRY(record(ev, 3, stream));
   HKV_TRY(launch_topp<true>(sh, c, ws, L, a->tau, a->p, a->select_mode, a->mask, stream));
   HKV_TRY(record(ev, 4, stream));
