@@ -34,7 +34,7 @@ def test_every_declared_function_is_exported(lib):
         assert hasattr(lib, n)
 
 
-def test_north_star_entry_points_declared():
+def test_hot_path_entry_points_declared():
     for n in ("hardkv_append", "hardkv_score_calibrate_topp", "hardkv_regularize",
               "hardkv_condense", "hardkv_decode_attn"):
         assert n in B.header_functions()
