@@ -4,9 +4,10 @@
 // [Condensed slots 0..C). All units' lists are concatenated and cut into contiguous
 // ranges of equal cost, one per CTA (split-K that stays balanced for ragged lengths; a
 // row gathered from the ring costs 3, any other row 2, each unit segment 320).
-// Each of a CTA's four compute warps leaves one log-sum-exp partial per unit segment
-// the CTA covers; the last CTA to finish a segment of a unit (an atomic count, no
-// waiting) merges that unit's partials into the output. In fused mode the compact
+// A CTA's four compute warps keep their own online-softmax states; at the end of each
+// unit segment the CTA merges them into one log-sum-exp partial, and the last CTA to
+// finish a segment of a unit (an atomic count, no waiting) merges that unit's
+// partials into the output. In fused mode the compact
 // slots of units that reselected this step are gathered from the ring (positions from
 // sp_idx) and written to the compact layout in the same pass (HARD-KV technical
 // summary sec. 2.C Rewrite Cache), so kept rows are read once.

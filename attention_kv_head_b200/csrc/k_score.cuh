@@ -6,8 +6,8 @@
 // multi-stage mbarrier pipeline; two groups of four consumer warps take alternate
 // tiles, each warp 16 rows of a tile, and compute the (key x query) logits with
 // mma.sync m16n8k16 (keys in M, queries in N, one or two 8-query tiles), then max-pool
-// over the real queries. Work is split evenly over all
-// tiles of all units, so ragged sequence lengths stay balanced.
+// over the real queries. All units' tiles form one list, dealt to the CTAs round-robin
+// in chunks of kScoreChunk tiles, so ragged sequence lengths stay balanced.
 #pragma once
 #include "common.cuh"
 

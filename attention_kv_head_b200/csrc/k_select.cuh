@@ -8,7 +8,8 @@
 // two-level select finds the key theta of the last kept candidate of the (s desc,
 // position asc) order — the shortest prefix whose mass reaches p * Z or whose length
 // reaches Cap: a histogram over the distance below the max picks the bin where the
-// prefix ends, then a radix select over that bin's elements pins theta exactly.
+// prefix ends; that bin's elements are then ordered exactly (one warp's bitonic sort up
+// to 64 of them, a block-wide ranking up to 1024, a radix select beyond) to pin theta.
 #pragma once
 #include "common.cuh"
 #include "k_score.cuh"
