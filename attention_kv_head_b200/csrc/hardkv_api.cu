@@ -307,6 +307,33 @@ int resident_ctas(K kernel, int threads, size_t smem) {
   return n;
 }
 
+// resident_ctas remembered per (kernel, device, threads, shared-memory bytes), so a
+// persistent grid is sized once per configuration and never from another device's or
+// another batch size's figure; later calls (for instance during stream capture) only
+// read the table.
+template <typename K>
+int resident_ctas_cached(K kernel, int threads, size_t smem) {
+  struct Entry {
+    const void *fn;
+    int dev, threads;
+    size_t smem;
+    int n;
+  };
+  static Entry table[64];
+  static int n_table = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < n_table; ++i)
+    if (table[i].fn == (const void *)kernel && table[i].dev == dev && table[i].threads == threads &&
+        table[i].smem == smem)
+      return table[i].n;
+  const int n = resident_ctas(kernel, threads, smem);
+  if (n_table < 64) table[n_table++] = Entry{(const void *)kernel, dev, threads, smem, n};
+  return n;
+}
+
 int launch_append(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *k_new,
                   const void *v_new, void *ws, const Layout &L, cudaStream_t st) {
   int *counters = reinterpret_cast<int *>(static_cast<char *>(ws) + L.counters);
@@ -346,8 +373,7 @@ int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, cons
     HKV_TRY(make_kmap(&map, d, c.k_ring));
   const size_t smem = ScoreTma<D>::smem_bytes(sh.B);
   HKV_TRY(set_smem(score_tma_kernel<D, NT>, smem));
-  static int per_sm = 0;
-  if (!per_sm) per_sm = resident_ctas(score_tma_kernel<D, NT>, ScoreTma<D>::THREADS, smem);
+  const int per_sm = resident_ctas_cached(score_tma_kernel<D, NT>, ScoreTma<D>::THREADS, smem);
   const int grid = per_sm * device_sms();
   launch_pdl(score_tma_kernel<D, NT>, dim3(grid), dim3(ScoreTma<D>::THREADS), smem, st, sh, c,
              static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
@@ -457,6 +483,25 @@ int check_mode(int m) {
   return (m == HARDKV_SELECT_ALL || m == HARDKV_SELECT_MOVED) ? HARDKV_OK : HARDKV_EINVAL;
 }
 
+// Every check of a fused step's arguments. `host`: q, k_new, v_new, tau and out are host
+// buffers (copied or used in place; any alignment), mask is still a device pointer.
+int check_step_args(const hardkv_step_args *a, bool host) {
+  if (!a) return HARDKV_EINVAL;
+  if (host) {
+    if (!a->q || !a->k_new || !a->v_new || !a->out) return HARDKV_EINVAL;
+  } else {
+    HKV_TRY(check_ptr(a->q));
+    HKV_TRY(check_ptr(a->k_new));
+    HKV_TRY(check_ptr(a->v_new));
+    HKV_TRY(check_ptr(a->tau, true));
+    HKV_TRY(check_ptr(a->out));
+  }
+  HKV_TRY(check_ptr(a->mask, true));
+  HKV_TRY(check_p(a->p));
+  HKV_TRY(check_mode(a->select_mode));
+  return HARDKV_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------- entry points
@@ -528,15 +573,7 @@ int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const
 int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
                        const hardkv_step_args *a, void *ws, cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));
-  if (!a) return HARDKV_EINVAL;
-  HKV_TRY(check_ptr(a->q));
-  HKV_TRY(check_ptr(a->k_new));
-  HKV_TRY(check_ptr(a->v_new));
-  HKV_TRY(check_ptr(a->tau, true));
-  HKV_TRY(check_ptr(a->mask, true));
-  HKV_TRY(check_ptr(a->out));
-  HKV_TRY(check_p(a->p));
-  HKV_TRY(check_mode(a->select_mode));
+  HKV_TRY(check_step_args(a, false));
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
   const Layout L = layout(desc);
@@ -573,8 +610,9 @@ static void *mapped_host(const void *host) {
 
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
                             const hardkv_step_args *h, void *ws, cudaStream_t stream) {
+  // every argument is checked before the first copy is enqueued
   HKV_TRY(check_common(desc, cache, ws));
-  if (!h || !h->q || !h->k_new || !h->v_new || !h->out) return HARDKV_EINVAL;
+  HKV_TRY(check_step_args(h, true));
   const Layout L = layout(desc);
   const size_t e = elem_size(desc);
   const size_t U = (size_t)desc->batch * desc->n_kv_heads;

@@ -34,8 +34,8 @@ _M2 = np.uint64(0x94D049BB133111EB)
 _MASK64 = (1 << 64) - 1
 
 # tensor tags (arbitrary distinct constants)
-TAG_K, TAG_V, TAG_Q, TAG_TEMP, TAG_LEN, TAG_SPIKE, TAG_SPIKE_NOISE, TAG_MASK = (
-    0x4B, 0x56, 0x51, 0x54, 0x4C, 0x53, 0x4E, 0x4D)
+TAG_K, TAG_V, TAG_Q, TAG_TEMP, TAG_LEN, TAG_SPIKE, TAG_SPIKE_NOISE, TAG_MASK, TAG_TAU = (
+    0x4B, 0x56, 0x51, 0x54, 0x4C, 0x53, 0x4E, 0x4D, 0x43)
 
 F32, BF16 = "f32", "bf16"
 EVICT, MERGE = 0, 1
@@ -222,6 +222,17 @@ def temperature(w: Workload, b: int, h: int) -> float:
     lo, hi = w.temp_range
     u = float(uniform(stream_key(w.seed, TAG_TEMP, b, h), np.zeros(1, np.uint64))[0])
     return float(np.float32(math.exp(math.log(lo) + u * (math.log(hi) - math.log(lo)))))
+
+
+def calibration_taus(w: Workload, lo: float = 0.25, hi: float = 8.0) -> np.ndarray:
+    """Caller-supplied calibration temperatures tau[b, h] (float32) for tests of the
+    temperature path: log-uniform in [lo, hi] per (sequence, KV head), so values fall on
+    both sides of 1, with unit (0, 0) exactly 1."""
+    B, H = w.batch, w.n_kv_heads
+    u = uniform(stream_key(w.seed, TAG_TAU), np.arange(B * H, dtype=np.uint64)).reshape(B, H)
+    t = np.exp(math.log(lo) + u * (math.log(hi) - math.log(lo))).astype(np.float32)
+    t[0, 0] = 1.0
+    return t
 
 
 def query_f32(w: Workload, step: int, b: int, qh: int) -> np.ndarray:

@@ -6,10 +6,12 @@ A step is one pass of the whole hot path (append, condense on block steps, score
 calibration + top-p, regularize fused with attention, combine) over one batch of
 synthetic input, replayed from the same starting cache state so every timed step is
 the workload's single decode step. Each step is one CUDA-graph replay timed with CUDA
-events on the launching stream; L2 is flushed (a 2 x L2 write) before every timed
-step, outside the timed events. `e2e` repeats the measurement through the host-buffer
-C entry point (hardkv_decode_step_host: pinned H2D of q / k_new / v_new, the step,
-D2H of the output). With --gpus N (torchrun) every rank runs an independent replica of
+events on the launching stream; L2 is flushed before every timed step, outside the
+timed events: a 2 x L2 buffer is written and then read back, so no line of the
+previous step survives and the flush's own dirty lines are written back before the
+timed region starts (the L2 is left holding clean lines of the flush buffer). `e2e`
+repeats the measurement through the host-buffer C entry point
+(hardkv_decode_step_host: pinned H2D of q / k_new / v_new, the step, D2H of the output). With --gpus N (torchrun) every rank runs an independent replica of
 the workload on its own GPU (no collective in the step) and the step time is the max
 over ranks.
 
@@ -215,6 +217,10 @@ def run_gpu(args, world, rank, local) -> dict:
     mask = dc.new_mask()
     snap = dc.snapshot_bounds()
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush_l2():
+        flush.zero_()                      # write 2 x L2 ...
+        flush.view(torch.int32).sum()      # ... then read it back: clean lines only
     stream = torch.cuda.Stream(device=dev)
     evs = [torch.cuda.Event(enable_timing=True) for _ in range(Bn.STEP_EVENTS)]
     with torch.cuda.stream(stream):
@@ -242,7 +248,7 @@ def run_gpu(args, world, rank, local) -> dict:
     def one_step(graph):
         with torch.cuda.stream(stream):
             dc.restore_bounds(snap)
-            flush.zero_()
+            flush_l2()
             t0.record(stream)
             graph.replay()
             t1.record(stream)
@@ -278,7 +284,7 @@ def run_gpu(args, world, rank, local) -> dict:
     for i in range(args.warmup + args.steps):
         with torch.cuda.stream(stream):
             dc.restore_bounds(snap)
-            flush.zero_()
+            flush_l2()
             t0 = torch.cuda.Event(enable_timing=True)
             t1 = torch.cuda.Event(enable_timing=True)
             t0.record(stream)
@@ -298,38 +304,34 @@ def run_gpu(args, world, rank, local) -> dict:
 
 # ----------------------------------------------------------------------------- oracle
 
-_ORACLE_CACHE: dict = {}
-
-
-def oracle_inputs(w):
-    """Per-unit exact inputs of the workload's first decode step (generated once)."""
-    if w.name in _ORACLE_CACHE:
-        return _ORACLE_CACHE[w.name]
+def _oracle_unit_inputs(w, unit_ids):
+    """Exact per-unit inputs of the workload's first decode step for the given units."""
     from attention_kv_head_b200 import synth
     lens = synth.seq_lengths(w)
     _, q_ex = synth.queries(w, 0)
     _, k_ex, _, v_ex = synth.step_kv(w, lens, 0)
     G = w.group
-    units = []
-    for b in range(w.batch):
+    out = []
+    for u in unit_ids:
+        b, h = divmod(u, w.n_kv_heads)
         L0 = int(lens[b]) - 1
-        for h in range(w.n_kv_heads):
-            _, ke, _, ve = synth.unit_kv(w, b, h, 0, L0)
-            units.append((b, h, L0, ke, ve, q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h]))
-    _ORACLE_CACHE[w.name] = units
-    return units
+        _, ke, _, ve = synth.unit_kv(w, b, h, 0, L0)
+        out.append((b, h, L0, ke, ve, q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h]))
+    return out
 
 
-def oracle_timing(w, budget_s: float) -> dict:
-    """Time the oracle's decode step on whole steps (all (sequence, KV-head) units of the
-    workload's first step) repeated until `budget_s` of oracle time; at least one unit."""
+def _oracle_worker(task):
+    """One pool process: time whole (sequence, KV-head) unit steps of the oracle on its
+    share of the units until `budget_s` of oracle time has run."""
+    name, seed, unit_ids, budget_s = task
     from attention_kv_head_b200 import synth
     from oracle import hardkv_oracle as O
+    w = synth.WORKLOADS[name].with_(seed=seed)
     p = synth.p_values(w)[0]
     prm = O.Params(w.head_dim, w.group, w.dense_window, w.condensed_slots, w.block,
                    w.sparse_cap, w.n_sink, w.dtype, w.condense_mode)
     C = w.condensed_slots
-    units = oracle_inputs(w)
+    units = _oracle_unit_inputs(w, unit_ids)
     done, elapsed = 0, 0.0
     while elapsed < budget_s:
         for (b, h, L0, ke, ve, qg, kx, vx) in units:
@@ -341,16 +343,59 @@ def oracle_timing(w, budget_s: float) -> dict:
             done += 1
             if elapsed >= budget_s:
                 break
-    step_s = elapsed / done * len(units)
+    return done, elapsed
+
+
+class OraclePool:
+    """The fp64 oracle as it stands, run over the workload's independent (sequence,
+    KV-head) units by a pool of single-threaded processes, one per host core this
+    process may use (spawned, so it is safe after CUDA has been initialised)."""
+
+    def __init__(self, w):
+        import multiprocessing as mp
+        self.w = w
+        self.workers = max(1, min(len(os.sched_getaffinity(0)), w.units))
+        saved = {k: os.environ.get(k) for k in _BLAS_VARS}
+        for k in _BLAS_VARS:
+            os.environ[k] = "1"          # one BLAS thread per process: cores = processes
+        try:
+            self.pool = mp.get_context("spawn").Pool(self.workers)
+        finally:
+            for k, v in saved.items():
+                if v is None:
+                    os.environ.pop(k, None)
+                else:
+                    os.environ[k] = v
+        self.shares = [list(range(i, w.units, self.workers)) for i in range(self.workers)]
+
+    def time(self, budget_s: float) -> dict:
+        w = self.w
+        res = self.pool.map(_oracle_worker, [(w.name, w.seed, sh, budget_s) for sh in self.shares])
+        done = sum(d for d, _ in res)
+        rate = sum(d / e for d, e in res if e > 0)      # unit steps per second, all processes
+        step_s = w.units / rate
+        return {"value": w.batch / step_s, "unit": "tokens/s", "cores": self.workers,
+                "kind": "oracle", "seconds": round(max(e for _, e in res), 3),
+                "sample": f"{done} (sequence, KV-head) unit steps of the {w.name} decode step "
+                          f"({w.units} units per step) run by {self.workers} single-threaded "
+                          f"processes for {budget_s:.1f} s each; step time = units per step / "
+                          f"summed unit-step rate"}
+
+    def close(self):
+        self.pool.close()
+        self.pool.join()
+
+
+_BLAS_VARS = ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")
+
+
+def oracle_timing(w, budget_s: float) -> dict:
+    """Time the oracle on the workload's first decode step for about `budget_s`."""
+    pool = OraclePool(w)
     try:
-        from threadpoolctl import threadpool_info
-        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = 1
-    return {"value": w.batch / step_s, "unit": "tokens/s", "cores": int(cores),
-            "kind": "oracle", "seconds": round(elapsed, 3),
-            "sample": f"{done} (sequence, KV-head) unit steps of the {w.name} decode step "
-                      f"({len(units)} units per step); step time = mean unit time x {len(units)}"}
+        return pool.time(budget_s)
+    finally:
+        pool.close()
 
 
 # ----------------------------------------------------------------------------- main
@@ -373,7 +418,7 @@ def main(argv=None):
               "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
               "dense_window": w.dense_window, "condensed_slots": w.condensed_slots,
               "sparse_cap": w.sparse_cap, "p": synth.p_values(w)[0],
-              "l2": "flushed (2 x L2 write) before every timed step",
+              "l2": "flushed before every timed step: 2 x L2 written, then read back",
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
     if args.impl == "reference":
@@ -381,10 +426,14 @@ def main(argv=None):
             return 0
         per_step = max(0.2, min(10.0, 60.0 / max(args.steps + args.warmup, 1)))
         vals, cb = [], None
-        for i in range(args.warmup + args.steps):
-            cb = oracle_timing(w, per_step)
-            if i >= args.warmup:
-                vals.append(cb["value"])
+        pool = OraclePool(w)
+        try:
+            for i in range(args.warmup + args.steps):
+                cb = pool.time(per_step)
+                if i >= args.warmup:
+                    vals.append(cb["value"])
+        finally:
+            pool.close()
         v = float(np.mean(vals))
         cb["value"] = v
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",

@@ -235,7 +235,9 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
  *    array; larger problems return HARDKV_ESCRATCH (nothing is enqueued).
  *  - The first call on a device looks up the array's device address with
  *    cudaGetSymbolAddress while that device is current; make that first call before
- *    any stream capture that includes this entry point.
+ *    any stream capture that includes this entry point. The address is then kept for
+ *    the life of the process: a caller that resets the device (cudaDeviceReset) must
+ *    not call this entry point on that device afterwards.
  *  - Every call, on every stream, shares the one array and leaves its contents there;
  *    nothing in it needs to start at zero (each call writes what it reads). Calls whose
  *    executions overlap on the GPU race on the array: serialise them (one stream, or

@@ -2,6 +2,9 @@
 oracle on the same seeded inputs, and compare them."""
 from __future__ import annotations
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -13,6 +16,23 @@ from oracle import hardkv_oracle as O
 # bf16 attention tolerance: max-abs 1e-2 and rel-L2 2e-3 (fixed by the target bounds);
 # fp32 inputs: the same arithmetic with fp32 storage -> 1e-4 / 1e-5.
 TOL = {"bf16": (1e-2, 2e-3), "f32": (1e-4, 1e-5)}
+
+# Merge slot choices: the kernel ranks cosines in fp32; for d = 128 the error of an
+# fp32 cosine is below d * 2^-24 ~ 7.6e-6, so a slot decision may legitimately differ
+# from the fp64 oracle only where the oracle's top-1/top-2 gap is under 1e-5. Such a
+# unit is followed no further (its Condensed state may then differ by design).
+MERGE_TIE = 1e-5
+
+
+def record(kind: str, **fields) -> None:
+    """Append one JSON record of parity counts (flips, clamps, near-ties) to the file
+    named by HARDKV_PARITY_RECORD, if that variable is set."""
+    path = os.environ.get("HARDKV_PARITY_RECORD")
+    if not path:
+        return
+    fields["kind"] = kind
+    with open(path, "a") as f:
+        f.write(json.dumps(fields, default=lambda x: x.item() if hasattr(x, "item") else str(x)) + "\n")
 
 
 def oracle_params(w: synth.Workload) -> O.Params:
@@ -57,31 +77,64 @@ def device_rows(t: torch.Tensor) -> np.ndarray:
 
 
 class StepCompare:
-    """Accumulates the comparison of one step over units."""
+    """Accumulates the comparison of one step (or run) over units."""
 
     def __init__(self, dtype):
         self.atol, self.rtol = TOL[dtype]
         self.flipped_units = 0
         self.flipped_tokens = 0
+        self.selections = 0
+        self.clamps = 0
         self.units = 0
+        self.flipped_attended = 0
         self.worst_abs = 0.0
         self.worst_rel = 0.0
 
     def selection(self, sel: O.Selection, p: float, gpu_kept: np.ndarray):
+        """The GPU's kept set must equal the oracle's up to the near-threshold flip rule;
+        returns True when they are identical."""
         ok, nd = O.allowed_flips(sel, p, gpu_kept)
         assert ok, f"mask differs beyond the flip rule ({nd} tokens)"
+        self.selections += 1
+        self.clamps += int(sel.clamped)
         if nd:
             self.flipped_units += 1
             self.flipped_tokens += nd
         return nd == 0
 
-    def attention(self, gpu: np.ndarray, ref: np.ndarray):
+    def attention(self, gpu: np.ndarray, ref: np.ndarray, flipped: bool = False):
         self.units += 1
+        self.flipped_attended += int(flipped)
         a = float(np.abs(gpu - ref).max())
         r = rel_l2(gpu, ref)
         self.worst_abs = max(self.worst_abs, a)
         self.worst_rel = max(self.worst_rel, r)
         assert a <= self.atol and r <= self.rtol, (a, r)
+
+    def summary(self) -> dict:
+        return dict(selections=self.selections, flipped_units=self.flipped_units,
+                    flipped_tokens=self.flipped_tokens, clamps=self.clamps,
+                    attention_units=self.units, attention_units_flipped=self.flipped_attended,
+                    worst_abs=self.worst_abs, worst_rel_l2=self.worst_rel)
+
+
+def adopt_selection(un: O.Unit, kept_local: np.ndarray) -> None:
+    """Make the oracle unit's Sparse set the given kept candidates (local indices, as
+    read from a GPU mask that O.allowed_flips accepted): the attention of a step whose
+    selection flipped a near-threshold token is evaluated on the GPU's mask, and a unit
+    that keeps its set across steps (select on move) carries that set on. Rows, order
+    and index come from the oracle's own arrays and O.regularize."""
+    L = un.d_lo - un.s_lo
+    mask = np.zeros(L, bool)
+    mask[np.asarray(kept_local, np.int64)] = True
+    pos = np.arange(un.s_lo, un.d_lo)
+    un.n, un.idx, un.sp_k, un.sp_v = O.regularize(
+        mask, pos, un.K[un.s_lo:un.d_lo], un.V[un.s_lo:un.d_lo], un.prm.sparse_cap)
+
+
+def tau_of(tau, b: int, h: int) -> float:
+    """Calibration temperature of unit (b, h): 1 when no array is given."""
+    return 1.0 if tau is None else float(tau[b, h])
 
 
 def run_unfused_step(dc: DecodeCache, q, k, v, p, select_mode=B.SELECT_ALL, tau=None):

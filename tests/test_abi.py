@@ -116,3 +116,33 @@ def test_entry_points_validate_before_any_launch(lib):
 def test_strerror(lib):
     for code in (B.OK, B.EINVAL, B.EALIGN, B.EDTYPE, B.ECAP, B.ECUDA, 12345):
         assert isinstance(B.strerror(code), str) and B.strerror(code)
+
+
+def test_host_entry_validates_before_any_copy(lib):
+    """hardkv_decode_step_host checks p, the select mode and the mask before its first
+    copy: a bad argument returns its own code (on a machine without a GPU a copy would
+    have failed with HARDKV_ECUDA instead)."""
+    import numpy as np
+    d = desc(batch=2, sparse_cap=100, ring_rows=1024, dense_window=64, condensed_slots=32)
+    c = _fake_cache()
+    ws = ctypes.c_void_p(0x7000000)
+    q = np.zeros((2, 32, 128), np.uint16)
+    kv = np.zeros((2, 8, 128), np.uint16)
+    out = np.zeros((2, 32, 128), np.float32)
+    tau = np.ones((2, 8), np.float32)
+
+    def call(p=0.9, mode=0, mask=None, tau_ptr=None):
+        a = B.StepArgs(q.ctypes.data, kv.ctypes.data, kv.ctypes.data, tau_ptr, ctypes.c_float(p),
+                       mode, mask, out.ctypes.data, None)
+        return lib.hardkv_decode_step_host(ctypes.byref(d), ctypes.byref(c), ctypes.byref(a), ws,
+                                           None)
+
+    for p in (0.0, 1.5, float("nan")):
+        assert call(p=p) == B.EINVAL
+        assert call(p=p, tau_ptr=tau.ctypes.data) == B.EINVAL
+    assert call(mode=7) == B.EINVAL
+    assert call(mask=0x1004) == B.EALIGN
+    a = B.StepArgs(None, kv.ctypes.data, kv.ctypes.data, None, ctypes.c_float(0.9), 0, None,
+                   out.ctypes.data, None)
+    assert lib.hardkv_decode_step_host(ctypes.byref(d), ctypes.byref(c), ctypes.byref(a), ws,
+                                       None) == B.EINVAL

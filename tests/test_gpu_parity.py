@@ -53,7 +53,10 @@ SMALL = {
 }
 
 
-def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_expected=None):
+def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, tau=None):
+    """Steps every oracle unit once and checks the GPU's step against it: boundaries,
+    mask (flip rule), compaction of the GPU's own mask bit-exact, attention on the GPU's
+    mask for every unit (a flipped unit's oracle set is the GPU's accepted one)."""
     G = w.group
     m = mask.cpu().numpy().view(np.uint32)
     n_kept = dc.n_kept.cpu().numpy()
@@ -64,8 +67,8 @@ def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_ex
     lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
     results = {}
     for (b, h), unit in units.items():
-        res = unit.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, p)
-        results[b, h] = res
+        qg = q_ex[b, h * G:(h + 1) * G]
+        res = unit.step(qg, k_ex[b, h], v_ex[b, h], U.tau_of(tau, b, h), p)
         assert (lens[b], dlo[b], slo[b]) == (unit.len, unit.d_lo, unit.s_lo)
         L = unit.d_lo - unit.s_lo
         kept = U.mask_bits(m[b, h], L)
@@ -81,21 +84,24 @@ def compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, moved_ex
         same = cmp.selection(res.sel, p, kept) if res.sel is not None else True
         if same:
             assert n == res.n and np.array_equal(sp_idx[b, h], res.idx)
-            cmp.attention(o[b, h * G:(h + 1) * G], res.out)
-        results[b, h] = (res, same)
+            ref = res.out
+        else:
+            U.adopt_selection(unit, kept)
+            ref = unit.attend(qg)
+        cmp.attention(o[b, h * G:(h + 1) * G], ref, flipped=not same)
+        results[b, h] = (res, same, ref)
     return results
 
 
-@pytest.mark.parametrize("name", list(SMALL))
-def test_small_step_unfused_vs_oracle_and_fused(name):
-    w = SMALL[name]
+def run_small_step(name, w, tau_np):
     st = synth.initial_state(w)
     dc = DecodeCache.from_state(st)
     dc2 = DecodeCache.from_state(st)
     (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    tau = None if tau_np is None else torch.from_numpy(tau_np).to(dc.device)
     p = synth.p_values(w)[0]
-    mask, out = U.run_unfused_step(dc, q, k, v, p)
-    mask2, out2 = U.run_fused_step(dc2, q, k, v, p)
+    mask, out = U.run_unfused_step(dc, q, k, v, p, tau=tau)
+    mask2, out2 = U.run_fused_step(dc2, q, k, v, p, tau=tau)
     torch.cuda.synchronize()
     units = {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
              for h in range(w.n_kv_heads)}
@@ -109,7 +115,7 @@ def test_small_step_unfused_vs_oracle_and_fused(name):
         got = sc[b * w.n_kv_heads + h, :L]
         assert np.allclose(got, ref, rtol=1e-5, atol=1e-5 * np.abs(ref).max()), name
     cmp = U.StepCompare(w.dtype)
-    results = compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp)
+    results = compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, p, cmp, tau=tau_np)
     # fused step == unfused path (selection, compaction and bookkeeping bit for bit)
     assert torch.equal(mask, mask2)
     assert torch.equal(dc.n_kept, dc2.n_kept) and torch.equal(dc.sp_idx, dc2.sp_idx)
@@ -120,17 +126,35 @@ def test_small_step_unfused_vs_oracle_and_fused(name):
         for h in range(w.n_kv_heads):
             assert torch.equal(dc.k_sp[b, h, :n[b, h]], dc2.k_sp[b, h, :n[b, h]])
             assert torch.equal(dc.v_sp[b, h, :n[b, h]], dc2.v_sp[b, h, :n[b, h]])
-    # the fused path splits the work by cost (gathered rows weigh two), the standalone
+    # the fused path splits the work by cost (gathered rows weigh more), the standalone
     # attention by rows: same math, different split-K summation order, so the fused
-    # output is held to the oracle bound itself
+    # output is held to the oracle bound itself (on the same, GPU-chosen mask)
     o2 = out2.cpu().numpy()
-    for (b, h), (res, same) in results.items():
-        if same:
-            cmp.attention(o2[b, h * w.group:(h + 1) * w.group], res.out)
+    for (b, h), (res, same, ref) in results.items():
+        cmp.attention(o2[b, h * w.group:(h + 1) * w.group], ref, flipped=not same)
     st_words = dc.read_status()
     assert st_words[B.ST_FLAGS] == 0
     assert st_words[B.ST_SELECTIONS] == w.units
-    print(name, "flipped units", cmp.flipped_units, "worst abs", cmp.worst_abs, "rel", cmp.worst_rel)
+    # clamps counted on the device = the oracle's (a flip at the boundary may move one)
+    assert abs(int(st_words[B.ST_CLAMPS]) - cmp.clamps) <= cmp.flipped_units
+    U.record("small_step", name=name, tau=tau_np is not None, **cmp.summary())
+    print(name, "tau" if tau_np is not None else "", cmp.summary())
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_small_step_unfused_vs_oracle_and_fused(name):
+    run_small_step(name, SMALL[name], None)
+
+
+TAU_CASES = ["bf16_d128_g4", "f32_d64_g1", "bf16_g16", "clamp", "p_low", "batch5", "keep_all_clamped"]
+
+
+@pytest.mark.parametrize("name", TAU_CASES)
+def test_small_step_with_calibration_temperatures(name):
+    """Caller-supplied temperatures tau[b,h] log-uniform in [0.25, 8] (unit (0,0) = 1)
+    drive the calibration softmax(s / tau) of both the separate and the fused path."""
+    w = SMALL[name]
+    run_small_step(name, w, synth.calibration_taus(w))
 
 
 @pytest.mark.parametrize("frac,cap", [(0.3, 600), (0.9, 200), (0.0, 600), (1.0, 600)])
@@ -251,38 +275,49 @@ def test_multistep_small(mode, select):
             res = un.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, w.p, reselect=rs)
             assert (bounds[0][b], bounds[1][b], bounds[2][b], bool(bounds[3][b])) == \
                 (un.len, un.d_lo, un.s_lo, res.moved)
-            if res.merge is not None and res.merge.gaps and min(res.merge.gaps) <= 1e-6:
+            if res.merge is not None and res.merge.gaps and min(res.merge.gaps) <= U.MERGE_TIE:
                 diverged.add((b, h))      # a near-tie may legitimately pick another slot
                 continue
             assert np.array_equal(w_cd[b, h], un.cd_w.astype(np.float32))
             assert np.array_equal(k_cd[b, h], un.cd_k) and np.array_equal(v_cd[b, h], un.cd_v)
-            same = True
+            same, ref = True, res.out
             if res.sel is not None:
                 L = un.d_lo - un.s_lo
-                same = cmp.selection(res.sel, w.p, U.mask_bits(m[b, h], L))
-            if same:
-                assert n_kept[b, h] == un.n and np.array_equal(sp_idx[b, h], un.idx)
-                cmp.attention(o[b, h * G:(h + 1) * G], res.out)
+                kept = U.mask_bits(m[b, h], L)
+                same = cmp.selection(res.sel, w.p, kept)
+                if not same:          # carry the accepted GPU set on (select on move keeps it)
+                    U.adopt_selection(un, kept)
+                    ref = un.attend(q_ex[b, h * G:(h + 1) * G])
+            assert n_kept[b, h] == un.n and np.array_equal(sp_idx[b, h], un.idx)
+            cmp.attention(o[b, h * G:(h + 1) * G], ref, flipped=not same)
     assert dc.read_status()[B.ST_FLAGS] == 0
     assert len(diverged) <= 1
+    U.record("multistep_small", mode=mode, select=select, diverged=len(diverged), **cmp.summary())
 
 
+@pytest.mark.parametrize("with_tau", [False, True], ids=["tau1", "tau"])
 @pytest.mark.parametrize("name", ["pr1", "llama8b_8k"])
-def test_full_size_single_step(name):
-    """The single-step workloads at full size, every unit against the oracle."""
+def test_full_size_single_step(name, with_tau):
+    """The single-step workloads at full size, every unit against the oracle; with_tau:
+    caller-supplied calibration temperatures log-uniform in [0.25, 8]."""
     w = synth.WORKLOADS[name]
     st = synth.initial_state(w)
     dc = DecodeCache.from_state(st)
     (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
-    mask, out = U.run_fused_step(dc, q, k, v, w.p)
+    tau_np = synth.calibration_taus(w) if with_tau else None
+    tau = None if tau_np is None else torch.from_numpy(tau_np).to(dc.device)
+    mask, out = U.run_fused_step(dc, q, k, v, w.p, tau=tau)
     torch.cuda.synchronize()
     units = {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
              for h in range(w.n_kv_heads)}
     cmp = U.StepCompare(w.dtype)
-    compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, w.p, cmp)
+    compare_step(w, st, dc, mask, out, units, q_ex, k_ex, v_ex, w.p, cmp, tau=tau_np)
     assert cmp.flipped_units <= max(1, w.units // 50)
-    print(name, "flipped", cmp.flipped_units, cmp.flipped_tokens, "abs", cmp.worst_abs,
-          "rel", cmp.worst_rel, "kept", dc.n_kept.sum().item())
+    status = dc.read_status()
+    assert status[B.ST_FLAGS] == 0
+    U.record("full_size", workload=name, tau=with_tau, kept=int(dc.n_kept.sum().item()),
+             device_clamps=int(status[B.ST_CLAMPS]), **cmp.summary())
+    print(name, with_tau, cmp.summary(), "kept", dc.n_kept.sum().item())
 
 
 def test_graph_capture_replays_the_step():
@@ -317,18 +352,33 @@ def test_graph_capture_replays_the_step():
 
 @pytest.mark.parametrize("pinned", [(1, 1, 1, 1), (0, 0, 0, 0), (1, 1, 0, 1), (0, 1, 1, 0)],
                          ids=["pinned", "pageable", "mixed_kv", "mixed_out"])
-def test_host_entry_point_matches_device_step(pinned):
+@pytest.mark.parametrize("with_tau", [False, True], ids=["tau1", "tau"])
+def test_host_entry_point_matches_device_step(pinned, with_tau):
     """Host buffers: pinned mapped ones are used in place by the kernels, pageable ones
-    are staged by copies; every combination gives the device step's result."""
+    are staged by copies (tau always is); every combination gives the device step's
+    result."""
     w = synth.small(batch=2)
     st = synth.initial_state(w)
     dc = DecodeCache.from_state(st)
     dc2 = DecodeCache.from_state(st)
     (q, k, v), _ = U.upload_step(dc, w, st, 0)
-    _, out = U.run_fused_step(dc, q, k, v, w.p)
+    tau_np = synth.calibration_taus(w) if with_tau else None
+    tau = None if tau_np is None else torch.from_numpy(tau_np).to(dc.device)
+    mask = dc.new_mask()
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+    dc.step(q, k, v, out, w.p, tau=tau, mask=mask)
     host = [t.cpu() for t in (q, k, v)] + [torch.full(out.shape, float("nan"))]
     qh, kh, vh, oh = (t.pin_memory() if pn else t for t, pn in zip(host, pinned))
-    dc2.step_host(qh, kh, vh, oh, w.p)
+    tau_h = None if tau_np is None else torch.from_numpy(tau_np.copy())
+    mask2 = dc2.new_mask()
+    dc2.step_host(qh, kh, vh, oh, w.p, tau=tau_h, mask=mask2)
     torch.cuda.synchronize()
     assert torch.equal(oh, out.cpu())
+    assert torch.equal(mask2, mask)
     assert torch.equal(dc2.len, dc.len) and torch.equal(dc2.sp_idx, dc.sp_idx)
+    if with_tau:   # the temperatures changed the selection (they are not all 1)
+        dc3 = DecodeCache.from_state(st)
+        mask3 = dc3.new_mask()
+        dc3.step(q, k, v, torch.empty_like(out), w.p, mask=mask3)
+        torch.cuda.synchronize()
+        assert not torch.equal(mask3, mask)

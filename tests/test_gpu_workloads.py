@@ -21,21 +21,29 @@ if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
 
-def sample_units(w, st, k=3):
-    """A spread of units: first, last, middle; for ragged batches the shortest and
-    longest sequences too."""
+def sample_units(w, st, k=16):
+    """At least k units: first, last, middle; the units with the lowest and highest key
+    temperature (flattest and most peaked scores: the most and the fewest kept, so the
+    clamp and the threshold extremes); for ragged batches the shortest and longest
+    sequences; the rest seeded-random."""
     B_, H = w.batch, w.n_kv_heads
     picks = [(0, 0), (B_ - 1, H - 1), (B_ // 2, H // 2)]
+    temps = np.array([[synth.temperature(w, b, h) for h in range(H)] for b in range(B_)])
+    order = np.argsort(temps, axis=None)
+    for flat in order[:3].tolist() + order[-3:].tolist():
+        picks.append(divmod(int(flat), H))
     if w.context is None:
         picks += [(int(np.argmin(st.lens)), 1 % H), (int(np.argmax(st.lens)), 2 % H)]
-    return list(dict.fromkeys(picks))[:max(k, len(picks))]
+    rng = np.random.default_rng(1234)
+    picks = list(dict.fromkeys(picks))
+    while len(picks) < k:
+        bh = (int(rng.integers(B_)), int(rng.integers(H)))
+        if bh not in picks:
+            picks.append(bh)
+    return picks
 
 
-# Merge slot choices: the kernel ranks cosines in fp32; for d = 128 the error of an
-# fp32 cosine is below d * 2^-24 ~ 7.6e-6, so a slot decision may legitimately differ
-# from the fp64 oracle only where the oracle's top-1/top-2 gap is under 1e-5. Such a
-# unit is followed no further (its Condensed state may then differ by design).
-MERGE_TIE = 1e-5
+MERGE_TIE = U.MERGE_TIE
 
 
 _STATES: dict = {}
@@ -57,7 +65,8 @@ def run_and_compare(w, p, select_on_move):
     cmp = U.StepCompare(w.dtype)
     G, H = w.group, w.n_kv_heads
     diverged = set()
-    moves = merged = 0
+    flips_per_unit = {}
+    moves = merged = ties = 0
     rows = torch.tensor([b * H + h for (b, h) in picks], device=dc.device)
     flat = lambda x: x.reshape(w.batch * H, *x.shape[2:]).index_select(0, rows).cpu()
     for t in range(w.steps):
@@ -85,19 +94,26 @@ def run_and_compare(w, p, select_on_move):
             moves += int(res.moved)
             if res.merge is not None and res.merge.gaps:
                 merged += len(res.merge.gaps)
+                ties += sum(g_ <= MERGE_TIE for g_ in res.merge.gaps)
                 if min(res.merge.gaps) <= MERGE_TIE:
                     diverged.add((b, h))
                     continue
             assert np.array_equal(w_cd[i], un.cd_w.astype(np.float32)), (t, b, h)
             assert np.array_equal(k_cd[i], un.cd_k), (t, b, h)
             assert np.array_equal(v_cd[i], un.cd_v), (t, b, h)
-            same = True
+            same, ref = True, res.out
             if res.sel is not None:
                 L = un.d_lo - un.s_lo
-                same = cmp.selection(res.sel, p, U.mask_bits(m[i], L))
-            if same:
-                assert n_kept[i] == un.n and np.array_equal(sp_idx[i], un.idx), (t, b, h)
-                cmp.attention(o[b, h * G:(h + 1) * G], res.out)
+                kept = U.mask_bits(m[i], L)
+                same = cmp.selection(res.sel, p, kept)
+                if not same:
+                    # the accepted GPU set becomes the unit's set: attention this step
+                    # is evaluated on it and a unit that keeps its set carries it on
+                    U.adopt_selection(un, kept)
+                    ref = un.attend(q_ex[b, h * G:(h + 1) * G])
+                    flips_per_unit[b, h] = flips_per_unit.get((b, h), 0) + 1
+            assert n_kept[i] == un.n and np.array_equal(sp_idx[i], un.idx), (t, b, h)
+            cmp.attention(o[b, h * G:(h + 1) * G], ref, flipped=not same)
     status = dc.read_status()
     assert status[B.ST_FLAGS] == 0, status
     # device counters against the final bookkeeping: every block move shifts d_lo by
@@ -111,6 +127,13 @@ def run_and_compare(w, p, select_on_move):
     if w.condense_mode == synth.MERGE:
         assert status[B.ST_MERGED] == H * w.block * n_moves.sum()
     assert len(diverged) <= len(picks) // 2
+    U.record("workload", workload=w.name, p=p, steps=w.steps, units_followed=len(picks),
+             oracle_moves=moves, oracle_merged_tokens=merged, oracle_merge_near_ties=ties,
+             diverged_after_near_tie=len(diverged),
+             device_clamps=int(status[B.ST_CLAMPS]), device_near_ties=int(status[B.ST_NEAR_TIES]),
+             device_selections=int(status[B.ST_SELECTIONS]),
+             flips_per_unit={f"{b},{h}": c for (b, h), c in flips_per_unit.items()},
+             **cmp.summary())
     print(w.name, p, "units", len(picks), "oracle moves", moves, "oracle merges", merged,
           "diverged", len(diverged), "flipped", cmp.flipped_units, cmp.flipped_tokens,
           "compared", cmp.units, "worst abs", cmp.worst_abs, "rel", cmp.worst_rel,
