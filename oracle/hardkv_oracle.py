@@ -28,6 +28,16 @@ every formula below is a stated reading, listed in the repository's design notes
   boundaries append at pos = len; len += 1; when len - d_lo >= W + block the block
              [d_lo, d_lo+block) moves Dense->Sparse and [s_lo, s_lo+block)
              moves Sparse->Condensed                               (sec. 2.A stages 1, 4)
+  entropy    tau_h solves H(softmax(s / tau)) = mean_g H(softmax_j(q_g . k_j / sqrt(d)))
+  -matched   over the candidates (bisection on ln tau): the calibrated distribution
+  tau        carries the raw attention's entropy     (sec. 2.A Tier 2 "budget based on
+             attention entropy"; sec. 2.B; sec. 3 "mapping onto the raw attention")
+  top-k      the k best scores, ties to the lower position: the fixed-budget
+             selection the pages compare against               (sec. 2.B, sec. 4)
+  MTI        per head, rewrite the kept rows or load them in place: rewrite when the
+             rewrite's one-off bytes cost less than the scattered-read surcharge over
+             the steps the layout lives, with budget thresholds L_lower / L_upper
+                                                                   (sec. 2.C trade-off)
 
 Parity pins: every function here is pinned by tests/test_oracle_pins.py against
 closed forms, library routines, brute force on tiny inputs and invariants.
@@ -173,6 +183,118 @@ def allowed_flips(sel: Selection, p: float, gpu_kept: np.ndarray, eps: float = 1
         if not (abs(sel.probs[j] - pth) <= eps or rank[j] == edge):
             return False, int(diff.size)
     return True, int(diff.size)
+
+
+# ----------------------------------------------------------------------------
+# stage 2c': the fixed-budget alternative (top-k)
+# ----------------------------------------------------------------------------
+
+def top_k(scores: np.ndarray, k: int) -> Selection:
+    """Keep the min(k, L) candidates first in the (s desc, position asc) order: the
+    fixed-budget selection (the same k for every head) that the pages contrast with
+    calibrated top-p (sec. 2.B "Top-k vs. Top-p"; sec. 4 fixed-budget baselines).
+    Nothing is clamped: k is the budget itself."""
+    L = scores.size
+    order = np.lexsort((np.arange(L), -scores))
+    kk = min(int(k), L)
+    probs = calibrate(scores, 1.0)
+    return Selection(np.sort(order[:kk]), order, kk, kk, False, probs, np.cumsum(probs[order]))
+
+
+def allowed_flips_topk(scores: np.ndarray, sel: Selection, gpu_kept: np.ndarray,
+                       eps: float):
+    """Whether a top-k set chosen on lower-precision scores may differ from the oracle's:
+    the count must be the same, and every differing token's score must lie within `eps`
+    of the score of the oracle's last kept token (rank k), where rounding of the scores
+    can reorder it. Returns (ok, number of differing tokens)."""
+    L = scores.size
+    mine = np.zeros(L, bool)
+    mine[sel.kept] = True
+    theirs = np.zeros(L, bool)
+    theirs[np.asarray(gpu_kept, dtype=np.int64)] = True
+    diff = np.nonzero(mine ^ theirs)[0]
+    if diff.size == 0:
+        return True, 0
+    if theirs.sum() != sel.k or sel.k == 0:
+        return False, int(diff.size)
+    s_theta = scores[sel.order[sel.k - 1]]
+    return bool(np.all(np.abs(scores[diff] - s_theta) <= eps)), int(diff.size)
+
+
+# ----------------------------------------------------------------------------
+# stage 2b': entropy-matched Logits Calibration
+# ----------------------------------------------------------------------------
+
+def entropy(probs: np.ndarray) -> float:
+    """Shannon entropy -sum p ln p (nats) of a probability vector (0 ln 0 = 0)."""
+    p = probs[probs > 0]
+    return float(-(p * np.log(p)).sum())
+
+
+def attention_entropy(q_group: np.ndarray, k_rows: np.ndarray) -> float:
+    """Mean over the group's queries g of the entropy of the raw attention of q_g over
+    the candidate rows: H(softmax_j(q_g . k_j / sqrt(d))). The target of the
+    entropy-matched calibration (sec. 2.A Tier 2: a head-adaptive budget based on
+    the attention entropy)."""
+    if k_rows.shape[0] == 0:
+        return 0.0
+    d = q_group.shape[1]
+    logits = k_rows @ q_group.T / math.sqrt(d)          # [L, G]
+    return float(np.mean([entropy(calibrate(logits[:, g], 1.0))
+                          for g in range(q_group.shape[0])]))
+
+
+TAU_MIN, TAU_MAX = 2.0 ** -6, 2.0 ** 6
+
+
+def entropy_matched_tau(scores: np.ndarray, target: float, iters: int = 200) -> float:
+    """The temperature tau in [TAU_MIN, TAU_MAX] with H(softmax(s / tau)) = target.
+
+    Reading of sec. 2.B ("maps the distribution of a selection strategy onto a
+    normalised softmax by adjusting the temperature ... preserving order") and sec. 3
+    ("mapping the distribution alteration onto the raw attention distribution"): the
+    temperature is chosen so that the calibrated distribution of the importance scores
+    has the entropy of the raw attention. H(softmax(s/tau)) grows with tau, so the root
+    is found by bisection on ln tau; the ends of the range are returned when the target
+    lies outside what the range can reach. No candidates or one candidate: tau = 1."""
+    if scores.size <= 1:
+        return 1.0
+    lo, hi = math.log(TAU_MIN), math.log(TAU_MAX)
+    if entropy(calibrate(scores, TAU_MAX)) <= target:
+        return TAU_MAX
+    if entropy(calibrate(scores, TAU_MIN)) >= target:
+        return TAU_MIN
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        if entropy(calibrate(scores, math.exp(mid))) < target:
+            lo = mid
+        else:
+            hi = mid
+    return math.exp(0.5 * (lo + hi))
+
+
+# ----------------------------------------------------------------------------
+# stage 3 policy: Rewrite Cache or Sparse Loading (Memory-Time Integral)
+# ----------------------------------------------------------------------------
+
+def mti_rewrite(n: int, reuse_steps: int, l_lower: int, l_upper: int,
+                gather_surcharge: float, write_cost: float = 1.0) -> bool:
+    """True: rewrite the head's n kept rows into the compact layout; False: load them in
+    place from the raw rows through the flattened index (sec. 2.C: Rewrite Cache vs.
+    Sparse Loading, chosen per head by a Memory-Time Integral that weighs the one-off
+    rewrite against the per-step decode gain, with budget thresholds L_lower, L_upper).
+
+    Reading: a kept row costs 1 per byte to read from a contiguous layout and
+    1 + gather_surcharge per byte to read scattered; a rewrite costs write_cost per byte
+    once. Over the `reuse_steps` later steps that read the same selection, rewriting
+    pays when write_cost < reuse_steps * gather_surcharge (the row count n cancels).
+    Budgets below L_lower are always loaded in place, budgets above L_upper always
+    rewritten."""
+    if n < l_lower:
+        return False
+    if n > l_upper:
+        return True
+    return write_cost < reuse_steps * gather_surcharge
 
 
 # ----------------------------------------------------------------------------
@@ -327,11 +449,23 @@ class Unit:
                         self.cd_w, P.n_sink, P.dtype, log)
 
     # stages 2-3 --------------------------------------------------------------
-    def select(self, q_group: np.ndarray, tau: float, p: float) -> Selection:
+    def select(self, q_group: np.ndarray, tau: float, p: float, rule: str = "topp",
+               k: int | None = None, calibration: str = "tau") -> Selection:
+        """Score the Sparse candidates and keep a subset: rule "topp" = calibrated top-p
+        (calibration "tau": the given temperature; "entropy": the entropy-matched one),
+        rule "topk" = the k best scores. The temperature used is kept in self.tau."""
         P = self.prm
         pos = np.arange(self.s_lo, self.d_lo)
         s = score(q_group, self.K[self.s_lo:self.d_lo])
-        sel = top_p(s, tau, p, P.sparse_cap)
+        if rule == "topk":
+            sel = top_k(s, min(int(k), P.sparse_cap))
+        else:
+            if calibration == "entropy":
+                tau = entropy_matched_tau(
+                    s, attention_entropy(q_group, self.K[self.s_lo:self.d_lo]))
+            sel = top_p(s, tau, p, P.sparse_cap)
+        self.tau = tau
+        self.scores = s
         mask = np.zeros(pos.size, bool)
         mask[sel.kept] = True
         self.n, self.idx, self.sp_k, self.sp_v = regularize(
@@ -358,9 +492,11 @@ class Unit:
         K, V, bias = self.union()
         return attention(q_group, K, V, bias)
 
-    def step(self, q_group, k_new, v_new, tau: float, p: float, reselect: str = "all"):
+    def step(self, q_group, k_new, v_new, tau: float, p: float, reselect: str = "all",
+             rule: str = "topp", k: int | None = None, calibration: str = "tau"):
         """One decode step: append, condense (block steps), select (if this unit
-        reselects: "all" = every step, "moved" = on its block move), attend."""
+        reselects: "all" = every step, "moved" = on its block move; rule / k /
+        calibration as in select), attend."""
         moved = self.append(k_new, v_new)
         log = None
         if moved:
@@ -368,7 +504,7 @@ class Unit:
             self.condense(log)
         sel = None
         if reselect == "all" or (reselect == "moved" and moved):
-            sel = self.select(q_group, tau, p)
+            sel = self.select(q_group, tau, p, rule, k, calibration)
         out = self.attend(q_group)
         return StepOut(moved, sel is not None, sel, self.n, self.idx.copy(), out, log)
 

@@ -77,6 +77,53 @@ def _cosine_unnormalised(a, rows):
     return rows @ a
 
 
+def _attention_entropy_max(q_group, k_rows):
+    if k_rows.shape[0] == 0:
+        return 0.0
+    logits = k_rows @ q_group.T / math.sqrt(q_group.shape[1])
+    return float(max(O.entropy(O.calibrate(logits[:, g], 1.0)) for g in range(q_group.shape[0])))
+
+
+def _entropy_log2(probs):
+    p = probs[probs > 0]
+    return float(-(p * np.log2(p)).sum())
+
+
+def _entropy_matched_tau_inverted(scores, target, iters=200):
+    if scores.size <= 1:
+        return 1.0
+    lo, hi = math.log(O.TAU_MIN), math.log(O.TAU_MAX)
+    for _ in range(iters):
+        mid = 0.5 * (lo + hi)
+        if O.entropy(O.calibrate(scores, math.exp(mid))) > target:   # wrong direction
+            lo = mid
+        else:
+            hi = mid
+    return math.exp(0.5 * (lo + hi))
+
+
+def _top_k_position_desc(scores, k):
+    L = scores.size
+    order = np.lexsort((-np.arange(L), -scores))
+    kk = min(int(k), L)
+    probs = O.calibrate(scores, 1.0)
+    return O.Selection(np.sort(order[:kk]), order, kk, kk, False, probs, np.cumsum(probs[order]))
+
+
+def _top_k_one_more(scores, k):
+    return _orig_top_k(scores, k + 1)
+
+
+def _mti_le(n, reuse_steps, l_lower, l_upper, gather_surcharge, write_cost=1.0):
+    if n < l_lower:
+        return False
+    if n > l_upper:
+        return True
+    return write_cost <= reuse_steps * gather_surcharge
+
+
+_orig_top_k = O.top_k
+
 MUTANTS = [
     ("score", _score_no_scale, [lambda: P.test_score_brute_force(4, 16, 7)]),
     ("score", _score_min, [lambda: P.test_score_brute_force(4, 16, 7)]),
@@ -94,6 +141,14 @@ MUTANTS = [
     ("attention", _attention_no_scale, [P.test_attention_equals_torch_sdpa]),
     ("cosine", _cosine_unnormalised,
      [lambda: [P.test_merge_slot_choice_brute_force(s) for s in range(10)]]),
+    ("attention_entropy", _attention_entropy_max,
+     [P.test_attention_entropy_is_the_mean_of_the_queries_raw_entropies]),
+    ("entropy", _entropy_log2, [P.test_entropy_matches_scipy]),
+    ("entropy_matched_tau", _entropy_matched_tau_inverted,
+     [P.test_entropy_matched_tau_residual_scale_and_range]),
+    ("top_k", _top_k_position_desc, [lambda: [P.test_top_k_brute_force_small(s) for s in range(20)]]),
+    ("top_k", _top_k_one_more, [lambda: [P.test_top_k_brute_force_small(s) for s in range(20)]]),
+    ("mti_rewrite", _mti_le, [P.test_mti_policy_thresholds_and_break_even]),
 ]
 
 

@@ -451,3 +451,127 @@ def test_allowed_flips_rule():
     sel = O.top_p(s, 1.0, 0.875, 10)
     assert sel.k in (3, 4)
     assert O.allowed_flips(sel, 0.875, [0, 1, 2])[0] and O.allowed_flips(sel, 0.875, [0, 1, 2, 3])[0]
+
+
+# ---------------------------------------------------------------- top-k (fixed budget)
+
+@pytest.mark.parametrize("seed", range(20))
+def test_top_k_brute_force_small(seed):
+    """n <= 9: among all k-subsets exactly one holds every score at least as high as
+    every score left out, and takes the lowest positions among the scores tied at the
+    boundary; it is the oracle's."""
+    r = rng(300 + seed)
+    n = int(r.integers(1, 10))
+    s = np.round(r.normal(size=n), 1)          # coarse values: ties happen
+    for k in range(0, n + 2):
+        good = []
+        for sub in itertools.combinations(range(n), min(k, n)):
+            inn = np.zeros(n, bool)
+            inn[list(sub)] = True
+            if inn.all() or not inn.any():
+                good.append(sub)
+                continue
+            lo_in, hi_out = s[inn].min(), s[~inn].max()
+            if lo_in < hi_out:
+                continue
+            if lo_in == hi_out:   # boundary ties: kept ones must have the lower positions
+                tied_in = np.nonzero(inn & (s == lo_in))[0]
+                tied_out = np.nonzero(~inn & (s == lo_in))[0]
+                if tied_in.max() > tied_out.min():
+                    continue
+            good.append(sub)
+        assert len(good) == 1
+        sel = O.top_k(s, k)
+        assert sel.kept.tolist() == sorted(good[0]) and sel.k == min(k, n) and not sel.clamped
+
+
+def test_top_k_is_the_capacity_clamp_of_keep_all_and_ignores_monotone_maps():
+    s = rng(7).normal(size=300) * 2
+    for k in (1, 17, 150, 299, 300, 400):
+        ref = O.top_k(s, k).kept
+        assert np.array_equal(O.top_p(s, 1.0, 1.0, k).kept, ref)      # p = 1 clamped to k
+        assert np.array_equal(O.top_k(np.exp(s), k).kept, ref)        # order-only
+        assert np.array_equal(O.top_k(3 * s - 5, k).kept, ref)
+    assert O.top_k(s, 1).kept.tolist() == [int(np.argmax(s))]
+
+
+def test_allowed_flips_topk_rule():
+    s = np.array([5.0, 4.0, 3.0, 3.0 + 1e-9, 1.0])
+    sel = O.top_k(s, 3)
+    assert sel.kept.tolist() == [0, 1, 3]
+    assert O.allowed_flips_topk(s, sel, [0, 1, 3], 1e-6) == (True, 0)
+    assert O.allowed_flips_topk(s, sel, [0, 1, 2], 1e-6)[0]          # within eps of s_theta
+    assert not O.allowed_flips_topk(s, sel, [0, 1, 2], 1e-12)[0]
+    assert not O.allowed_flips_topk(s, sel, [0, 1, 4], 1e-6)[0]      # far from the boundary
+    assert not O.allowed_flips_topk(s, sel, [0, 1, 2, 3], 1e-6)[0]   # count must match
+
+
+# ---------------------------------------------------------------- entropy-matched calibration
+
+def test_entropy_matches_scipy():
+    for seed in range(5):
+        p = scipy.special.softmax(rng(400 + seed).normal(size=50) * 3)
+        assert abs(O.entropy(p) - scipy.stats.entropy(p)) < 1e-12
+    assert O.entropy(np.array([1.0, 0.0, 0.0])) == 0.0
+    assert abs(O.entropy(np.full(8, 1 / 8)) - math.log(8)) < 1e-12
+
+
+def test_attention_entropy_is_the_mean_of_the_queries_raw_entropies():
+    r = rng(11)
+    q = r.normal(size=(3, 16))
+    k = r.normal(size=(40, 16)) * 2
+    want = np.mean([scipy.stats.entropy(scipy.special.softmax(k @ q[g] / 4.0)) for g in range(3)])
+    assert abs(O.attention_entropy(q, k) - want) < 1e-12
+    assert abs(O.attention_entropy(q, np.zeros((40, 16))) - math.log(40)) < 1e-12
+    assert O.attention_entropy(q, np.zeros((0, 16))) == 0.0
+
+
+def test_entropy_matched_tau_single_query_is_one():
+    """G = 1: the max-pooled score is the raw logit, so the raw attention's entropy is
+    reached at tau = 1."""
+    r = rng(12)
+    for T in (0.5, 1.0, 3.0):
+        q = r.normal(size=(1, 64))
+        k = r.normal(size=(500, 64)) * T
+        s = O.score(q, k)
+        tau = O.entropy_matched_tau(s, O.attention_entropy(q, k))
+        assert abs(tau - 1.0) < 1e-9
+
+
+@pytest.mark.parametrize("sigma,target_drop", [(1.0, 0.2), (2.0, 0.5), (0.7, 0.05)])
+def test_entropy_matched_tau_gaussian_closed_form(sigma, target_drop):
+    """i.i.d. N(0, sigma^2) scores, large L: H(softmax(s/tau)) -> ln L - sigma^2/(2 tau^2)
+    (the softmax of N(0, v) logits tilts them to N(v, v): H = ln E[e^x] + ln L - E_p[x]),
+    so the target ln L - D is met at tau = sigma / sqrt(2 D)."""
+    L = 400000
+    s = rng(13).normal(size=L) * sigma
+    tau = O.entropy_matched_tau(s, math.log(L) - target_drop)
+    assert abs(tau / (sigma / math.sqrt(2 * target_drop)) - 1) < 0.02
+
+
+def test_entropy_matched_tau_residual_scale_and_range():
+    r = rng(14)
+    s = r.normal(size=2000) * 1.7
+    for target in (1.0, 3.0, 6.0, 7.5):
+        tau = O.entropy_matched_tau(s, target)
+        assert abs(O.entropy(O.calibrate(s, tau)) - target) < 1e-9
+        assert abs(O.entropy_matched_tau(4 * s, target) / tau - 4) < 1e-9     # scale equivariant
+    taus = [O.entropy_matched_tau(s, t) for t in (2.0, 4.0, 6.0)]
+    assert taus[0] < taus[1] < taus[2]                                          # monotone
+    assert O.entropy_matched_tau(s, math.log(s.size) + 1) == O.TAU_MAX         # unreachable
+    assert O.entropy_matched_tau(s, -1.0) == O.TAU_MIN
+    assert O.entropy_matched_tau(np.array([2.0]), 0.3) == 1.0
+
+
+# ---------------------------------------------------------------- MTI policy
+
+def test_mti_policy_thresholds_and_break_even():
+    # one-off write (1 per byte) against a 0.5 per byte scattered-read surcharge:
+    # rewriting pays once the selection is read in more than 2 later steps
+    assert not O.mti_rewrite(1000, 0, 64, 10 ** 6, 0.5)      # reselected every step
+    assert not O.mti_rewrite(1000, 2, 64, 10 ** 6, 0.5)      # 2 * 0.5 = 1: break-even, no gain
+    assert O.mti_rewrite(1000, 3, 64, 10 ** 6, 0.5)
+    assert O.mti_rewrite(1000, 15, 64, 10 ** 6, 0.5)
+    assert not O.mti_rewrite(10, 15, 64, 10 ** 6, 0.5)       # below L_lower: load in place
+    assert O.mti_rewrite(5000, 0, 64, 4096, 0.5)             # above L_upper: rewrite
+    assert O.mti_rewrite(64, 15, 64, 64, 0.5) and not O.mti_rewrite(63, 15, 64, 64, 0.5)
