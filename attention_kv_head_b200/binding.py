@@ -18,6 +18,8 @@ OK, EINVAL, EALIGN, EDTYPE, ECAP, ECUDA, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
 F32, BF16 = 0, 1
 EVICT, MERGE = 0, 1
 SELECT_ALL, SELECT_MOVED = 0, 1
+RULE_TOPP, RULE_TOPK = 0, 1
+CAL_TAU, CAL_ENTROPY = 0, 1
 STATUS_WORDS = 8
 ST_FLAGS, ST_CLAMPS, ST_NEAR_TIES, ST_MERGED, ST_MOVES, ST_SELECTIONS = range(6)
 DEV_RING_OVERFLOW, DEV_BAD_BOUNDS, DEV_SEGMENTS, DEV_WAIT_TIMEOUT = 1, 2, 4, 8
@@ -42,7 +44,8 @@ class Cache(ctypes.Structure):
 class StepArgs(ctypes.Structure):
     _fields_ = [("q", _vp), ("k_new", _vp), ("v_new", _vp), ("tau", _vp),
                 ("p", ctypes.c_float), ("select_mode", _i32), ("mask", _vp), ("out", _vp),
-                ("stage_events", _vp)]
+                ("stage_events", _vp), ("rule", _i32), ("top_k", _i32), ("calibration", _i32),
+                ("tau_out", _vp)]
 
 
 class HardKVError(RuntimeError):
@@ -61,6 +64,11 @@ _SIGS = {
     "hardkv_condense": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp]),
     "hardkv_score_calibrate_topp": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp,
                                                    _vp, ctypes.c_float, _i32, _vp, _vp, _vp]),
+    "hardkv_score_calibrate_entropy_topp": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),
+                                                           _vp, ctypes.c_float, _i32, _vp, _vp, _vp,
+                                                           _vp]),
+    "hardkv_score_topk": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _i32, _i32,
+                                         _vp, _vp, _vp]),
     "hardkv_regularize": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _i32,
                                          _vp, _vp]),
     "hardkv_decode_attn": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp,

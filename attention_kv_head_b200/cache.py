@@ -120,6 +120,15 @@ class DecodeCache:
         self._c("hardkv_score_calibrate_topp", _ptr(q), _ptr(tau), ctypes.c_float(p),
                 select_mode, _ptr(mask), _ptr(self.ws), _stream(stream))
 
+    def score_calibrate_entropy_topp(self, q, p, mask, tau_out=None, select_mode=B.SELECT_ALL,
+                                     stream=None):
+        self._c("hardkv_score_calibrate_entropy_topp", _ptr(q), ctypes.c_float(p), select_mode,
+                _ptr(mask), _ptr(tau_out), _ptr(self.ws), _stream(stream))
+
+    def score_topk(self, q, k, mask, select_mode=B.SELECT_ALL, stream=None):
+        self._c("hardkv_score_topk", _ptr(q), int(k), select_mode, _ptr(mask), _ptr(self.ws),
+                _stream(stream))
+
     def regularize(self, mask, select_mode=B.SELECT_ALL, stream=None):
         self._c("hardkv_regularize", _ptr(mask), select_mode, _ptr(self.ws), _stream(stream))
 
@@ -127,25 +136,28 @@ class DecodeCache:
         self._c("hardkv_decode_attn", _ptr(q), _ptr(out), _ptr(self.ws), _stream(stream))
 
     def step_args(self, q, k_new, v_new, out, p, tau=None, mask=None,
-                  select_mode=B.SELECT_ALL, events=None) -> B.StepArgs:
+                  select_mode=B.SELECT_ALL, events=None, rule=B.RULE_TOPP, top_k=0,
+                  calibration=B.CAL_TAU, tau_out=None) -> B.StepArgs:
         ev = None
         if events is not None:
             self._ev_arr = (ctypes.c_void_p * B.STEP_EVENTS)(
                 *[e.cuda_event if e is not None else None for e in events])
             ev = ctypes.cast(self._ev_arr, ctypes.c_void_p)
         return B.StepArgs(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(tau), ctypes.c_float(p),
-                          select_mode, _ptr(mask), _ptr(out), ev)
+                          select_mode, _ptr(mask), _ptr(out), ev, rule, int(top_k), calibration,
+                          _ptr(tau_out))
 
     def step(self, q, k_new, v_new, out, p, tau=None, mask=None, select_mode=B.SELECT_ALL,
-             events=None, stream=None):
-        """One fused decode step through hardkv_decode_step (device tensors)."""
-        args = self.step_args(q, k_new, v_new, out, p, tau, mask, select_mode, events)
+             events=None, stream=None, **sel):
+        """One fused decode step through hardkv_decode_step (device tensors); `sel` may
+        set rule / top_k / calibration / tau_out (hardkv_step_args)."""
+        args = self.step_args(q, k_new, v_new, out, p, tau, mask, select_mode, events, **sel)
         self._c("hardkv_decode_step", ctypes.byref(args), _ptr(self.ws), _stream(stream))
 
     def step_host(self, q, k_new, v_new, out, p, tau=None, mask=None, select_mode=B.SELECT_ALL,
-                  stream=None):
+                  stream=None, **sel):
         """hardkv_decode_step_host: q/k_new/v_new/tau/out are (pinned) host tensors."""
-        args = self.step_args(q, k_new, v_new, out, p, tau, mask, select_mode)
+        args = self.step_args(q, k_new, v_new, out, p, tau, mask, select_mode, **sel)
         self._c("hardkv_decode_step_host", ctypes.byref(args), _ptr(self.ws), _stream(stream))
 
     def read_status(self) -> np.ndarray:

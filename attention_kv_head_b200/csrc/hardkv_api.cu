@@ -101,7 +101,7 @@ Shape make_shape(const hardkv_desc *d) {
 }
 
 struct Layout {
-  size_t scores, tile_max, part, counters, st_q, st_k, st_v, st_out, st_tau, total;
+  size_t scores, tile_max, ent, part, counters, st_q, st_k, st_v, st_out, st_tau, total;
   int tm_stride, P;
 };
 
@@ -125,6 +125,7 @@ Layout layout(const hardkv_desc *d) {
   };
   L.scores = take(U * R * 4);
   L.tile_max = take(U * (size_t)L.tm_stride * 4);
+  L.ent = take(U * (size_t)L.tm_stride * G * kEntFloats * 4);
   L.part = take((size_t)L.P * kSegMax * G * (d->head_dim + kPartO) * 4);
   L.counters = take(U * 4);
   L.st_q = take((size_t)d->batch * d->n_q_heads * d->head_dim * e);
@@ -362,58 +363,85 @@ int launch_condense(const hardkv_desc *d, const Shape &sh, const Cache &c, cudaS
   return HARDKV_OK;
 }
 
-template <int D, int NT>
-int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
-                     float *scores, float *tm, int tm_stride, int select_mode, cudaStream_t st,
-                     const CUtensorMap *pre) {
+template <int D, int NT, bool ENT>
+int launch_score_tma_t(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
+                       const ScoreOut &so, int select_mode, cudaStream_t st, const CUtensorMap *pre) {
   CUtensorMap map;
   if (pre)
     map = *pre;
   else
     HKV_TRY(make_kmap(&map, d, c.k_ring));
   const size_t smem = ScoreTma<D>::smem_bytes(sh.B);
-  HKV_TRY(set_smem(score_tma_kernel<D, NT>, smem));
-  const int per_sm = resident_ctas_cached(score_tma_kernel<D, NT>, ScoreTma<D>::THREADS, smem);
+  HKV_TRY(set_smem(score_tma_kernel<D, NT, ENT>, smem));
+  const int per_sm = resident_ctas_cached(score_tma_kernel<D, NT, ENT>, ScoreTma<D>::THREADS, smem);
   const int grid = per_sm * device_sms();
-  launch_pdl(score_tma_kernel<D, NT>, dim3(grid), dim3(ScoreTma<D>::THREADS), smem, st, sh, c,
-             static_cast<const bf16 *>(q), scores, tm, tm_stride, select_mode, map);
+  launch_pdl(score_tma_kernel<D, NT, ENT>, dim3(grid), dim3(ScoreTma<D>::THREADS), smem, st, sh, c,
+             static_cast<const bf16 *>(q), so, select_mode, map);
   HKV_CHECK_LAUNCH("score_tma_kernel");
   return HARDKV_OK;
 }
 
+template <int D, int NT>
+int launch_score_tma(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q,
+                     const ScoreOut &so, int select_mode, cudaStream_t st, const CUtensorMap *pre) {
+  return so.ent ? launch_score_tma_t<D, NT, true>(d, sh, c, q, so, select_mode, st, pre)
+                : launch_score_tma_t<D, NT, false>(d, sh, c, q, so, select_mode, st, pre);
+}
+
+ScoreOut score_out(void *ws, const Layout &L, bool entropy) {
+  ScoreOut so;
+  so.scores = reinterpret_cast<float *>(static_cast<char *>(ws) + L.scores);
+  so.tile_max = reinterpret_cast<float *>(static_cast<char *>(ws) + L.tile_max);
+  so.ent = entropy ? reinterpret_cast<float *>(static_cast<char *>(ws) + L.ent) : nullptr;
+  so.tm_stride = L.tm_stride;
+  return so;
+}
+
 // `pre`: the key tensor map when the caller encoded it ahead of its first launch (the
 // fused step does, so no host work sits between its kernel launches); NULL: encode here.
+// `entropy`: also write the raw-attention entropy partials (entropy-matched calibration).
 int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *q, void *ws,
-                 const Layout &L, int select_mode, cudaStream_t st, const CUtensorMap *pre = nullptr) {
-  float *scores = reinterpret_cast<float *>(static_cast<char *>(ws) + L.scores);
-  float *tm = reinterpret_cast<float *>(static_cast<char *>(ws) + L.tile_max);
+                 const Layout &L, int select_mode, bool entropy, cudaStream_t st,
+                 const CUtensorMap *pre = nullptr) {
+  const ScoreOut so = score_out(ws, L, entropy);
   if (d->dtype == HARDKV_BF16) {
     if (sh.G <= 8)
-      return sh.d == 128 ? launch_score_tma<128, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre)
-                         : launch_score_tma<64, 1>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre);
-    return sh.d == 128 ? launch_score_tma<128, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre)
-                       : launch_score_tma<64, 2>(d, sh, c, q, scores, tm, L.tm_stride, select_mode, st, pre);
+      return sh.d == 128 ? launch_score_tma<128, 1>(d, sh, c, q, so, select_mode, st, pre)
+                         : launch_score_tma<64, 1>(d, sh, c, q, so, select_mode, st, pre);
+    return sh.d == 128 ? launch_score_tma<128, 2>(d, sh, c, q, so, select_mode, st, pre)
+                       : launch_score_tma<64, 2>(d, sh, c, q, so, select_mode, st, pre);
   }
   const dim3 grid(sh.R / kTile + 2, sh.B * sh.H);
   launch_pdl(score_f32_kernel, grid, dim3(128), (size_t)sh.G * sh.d * 4, st, sh, c,
-             static_cast<const float *>(q), scores, tm, L.tm_stride, select_mode);
+             static_cast<const float *>(q), so, select_mode);
   HKV_CHECK_LAUNCH("score_f32_kernel");
   return HARDKV_OK;
 }
 
 template <bool WRITE_IDX>
-int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, const float *tau,
-                float p, int select_mode, uint32_t *mask, cudaStream_t st) {
-  const float *scores = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.scores);
-  const float *tm = reinterpret_cast<const float *>(static_cast<char *>(ws) + L.tile_max);
+int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, const SelectParams &sp,
+                int select_mode, uint32_t *mask, cudaStream_t st) {
+  const ScoreOut so = score_out(ws, L, sp.ent != nullptr);
   // the unit's scores are cached in shared memory when a whole ring fits
   const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
   const size_t smem = topp_smem_bytes(cache_n);
   HKV_TRY(set_smem(topp_kernel<WRITE_IDX>, smem));
-  launch_pdl(topp_kernel<WRITE_IDX>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, scores, tm,
-             L.tm_stride, tau, p, select_mode, mask, cache_n);
+  launch_pdl(topp_kernel<WRITE_IDX>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, so, sp,
+             select_mode, mask, cache_n);
   HKV_CHECK_LAUNCH("topp_kernel");
   return HARDKV_OK;
+}
+
+SelectParams select_params(const float *tau, float p, int rule, int k, bool entropy, float *tau_out,
+                           void *ws, const Layout &L) {
+  SelectParams sp;
+  sp.tau = tau;
+  sp.ent = entropy ? reinterpret_cast<const float *>(static_cast<char *>(ws) + L.ent) : nullptr;
+  sp.tau_out = tau_out;
+  sp.p = p;
+  sp.rule = rule;
+  sp.k = k;
+  return sp;
 }
 
 AttendParams attend_params(const Shape &sh, const void *q, float *out, void *ws, const Layout &L,
@@ -479,6 +507,12 @@ int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const 
 }
 
 int check_p(float p) { return (p > 0.0f && p <= 1.0f) ? HARDKV_OK : HARDKV_EINVAL; }
+int check_rule(const hardkv_desc *d, int rule, int k, int calibration) {
+  if (rule != HARDKV_RULE_TOPP && rule != HARDKV_RULE_TOPK) return HARDKV_EINVAL;
+  if (rule == HARDKV_RULE_TOPK && (k < 1 || k > d->sparse_cap)) return HARDKV_EINVAL;
+  if (calibration != HARDKV_CAL_TAU && calibration != HARDKV_CAL_ENTROPY) return HARDKV_EINVAL;
+  return HARDKV_OK;
+}
 int check_mode(int m) {
   return (m == HARDKV_SELECT_ALL || m == HARDKV_SELECT_MOVED) ? HARDKV_OK : HARDKV_EINVAL;
 }
@@ -497,7 +531,8 @@ int check_step_args(const hardkv_step_args *a, bool host) {
     HKV_TRY(check_ptr(a->out));
   }
   HKV_TRY(check_ptr(a->mask, true));
-  HKV_TRY(check_p(a->p));
+  HKV_TRY(check_ptr(a->tau_out, true));
+  if (a->rule != HARDKV_RULE_TOPK) HKV_TRY(check_p(a->p));
   HKV_TRY(check_mode(a->select_mode));
   return HARDKV_OK;
 }
@@ -547,8 +582,45 @@ int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cac
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
   const Layout L = layout(desc);
-  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, stream));
-  return launch_topp<false>(sh, c, ws, L, tau, p, select_mode, mask, stream);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
+  return launch_topp<false>(sh, c, ws, L,
+                            select_params(tau, p, HARDKV_RULE_TOPP, 0, false, nullptr, ws, L),
+                            select_mode, mask, stream);
+}
+
+int hardkv_score_calibrate_entropy_topp(const hardkv_desc *desc, const hardkv_cache *cache,
+                                        const void *q, float p, int32_t select_mode,
+                                        uint32_t *mask, float *tau_out, void *ws,
+                                        cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(q));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_ptr(tau_out, true));
+  HKV_TRY(check_p(p));
+  HKV_TRY(check_mode(select_mode));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(cache);
+  const Layout L = layout(desc);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, true, stream));
+  return launch_topp<false>(sh, c, ws, L,
+                            select_params(nullptr, p, HARDKV_RULE_TOPP, 0, true, tau_out, ws, L),
+                            select_mode, mask, stream);
+}
+
+int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const void *q, int32_t k,
+                      int32_t select_mode, uint32_t *mask, void *ws, cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(q));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_rule(desc, HARDKV_RULE_TOPK, k, HARDKV_CAL_TAU));
+  HKV_TRY(check_mode(select_mode));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(cache);
+  const Layout L = layout(desc);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
+  return launch_topp<false>(sh, c, ws, L,
+                            select_params(nullptr, 1.0f, HARDKV_RULE_TOPK, k, false, nullptr, ws, L),
+                            select_mode, mask, stream);
 }
 
 int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache, const uint32_t *mask,
@@ -574,6 +646,8 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
                        const hardkv_step_args *a, void *ws, cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_step_args(a, false));
+  HKV_TRY(check_rule(desc, a->rule, a->top_k, a->calibration));
+  const bool entropy = a->rule == HARDKV_RULE_TOPP && a->calibration == HARDKV_CAL_ENTROPY;
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
   const Layout L = layout(desc);
@@ -586,9 +660,12 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(record(ev, 1, stream));
   HKV_TRY(launch_condense(desc, sh, c, stream));
   HKV_TRY(record(ev, 2, stream));
-  HKV_TRY(launch_score(desc, sh, c, a->q, ws, L, a->select_mode, stream, tma ? &kmap : nullptr));
+  HKV_TRY(launch_score(desc, sh, c, a->q, ws, L, a->select_mode, entropy, stream,
+                       tma ? &kmap : nullptr));
   HKV_TRY(record(ev, 3, stream));
-  HKV_TRY(launch_topp<true>(sh, c, ws, L, a->tau, a->p, a->select_mode, a->mask, stream));
+  HKV_TRY(launch_topp<true>(sh, c, ws, L,
+                            select_params(a->tau, a->p, a->rule, a->top_k, entropy, a->tau_out, ws, L),
+                            a->select_mode, a->mask, stream));
   HKV_TRY(record(ev, 4, stream));
   HKV_TRY(launch_attend(desc, sh, c, a->q, a->out, ws, L, 1, a->select_mode, false, stream));
   return record(ev, 5, stream);
@@ -613,6 +690,7 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   // every argument is checked before the first copy is enqueued
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_step_args(h, true));
+  HKV_TRY(check_rule(desc, h->rule, h->top_k, h->calibration));
   const Layout L = layout(desc);
   const size_t e = elem_size(desc);
   const size_t U = (size_t)desc->batch * desc->n_kv_heads;
@@ -725,8 +803,10 @@ int hardkv_score_calibrate_topp_static(const hardkv_desc *desc, const hardkv_cac
   HKV_TRY(static_scratch(&ws));
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
-  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, stream));
-  return launch_topp<false>(sh, c, ws, L, tau, p, select_mode, mask, stream);
+  HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
+  return launch_topp<false>(sh, c, ws, L,
+                            select_params(tau, p, HARDKV_RULE_TOPP, 0, false, nullptr, ws, L),
+                            select_mode, mask, stream);
 }
 
 }  // extern "C"

@@ -16,6 +16,17 @@ namespace hardkv {
 constexpr int kTile = 64;         // key rows per tile (ring rows are 64-aligned)
 constexpr int kPartsPerTile = 4;  // per-warp partial maxima per tile
 constexpr int kScoreChunk = 2;    // consecutive tiles a CTA takes before the next CTA
+constexpr int kEntFloats = 3;     // raw-attention entropy partial: (m, S0, S1) per query
+
+// Where the score stage writes: the fp32 scores [U][R] (candidate j of unit u at
+// u*R + j), per-part maxima [U][tm_stride] (part = 16 key rows of a tile) and, when the
+// entropy-matched calibration needs them (ent != nullptr), per-part raw-attention
+// partials [U][tm_stride][G][3]: for each query g of the group over the part's rows,
+// m = max l, S0 = sum exp(l - m), S1 = sum exp(l - m) (l - m), with l = q_g . k / sqrt(d).
+struct ScoreOut {
+  float *scores, *tile_max, *ent;
+  int tm_stride;
+};
 
 template <int D>
 struct ScoreTma {
@@ -68,11 +79,58 @@ __device__ __forceinline__ void load_qT_frags(uint32_t (&qb)[NT][D / 16][2], con
   }
 }
 
-template <int D, int NT>
+// Raw-attention entropy partials of one 16-row warp slice (rows g and g+8 of lane
+// (g, t); ok0 / ok8 = those rows are Sparse candidates) for the queries of the lane's
+// accumulator columns; lanes with g == 0 store them. All lanes must call it.
+template <int NT>
+__device__ __forceinline__ void entropy_partials(const float (&sa)[NT][4], const float (&sb)[NT][4],
+                                                 bool ok0, bool ok8, float scale, int G, int lane,
+                                                 float *ep) {
+  const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int qi = nt * 8 + 2 * t + e;
+      const float x0 = ok0 ? (sa[nt][e] + sb[nt][e]) * scale : -INFINITY;
+      const float x8 = ok8 ? (sa[nt][2 + e] + sb[nt][2 + e]) * scale : -INFINITY;
+      float m = fmaxf(x0, x8);
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+      float s0 = 0.f, s1 = 0.f;
+      if (m != -INFINITY) {
+        if (ok0) {
+          const float dd = x0 - m, ee = expf(dd);
+          s0 += ee;
+          s1 += ee * dd;
+        }
+        if (ok8) {
+          const float dd = x8 - m, ee = expf(dd);
+          s0 += ee;
+          s1 += ee * dd;
+        }
+      }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+      }
+      if (g == 0 && qi < G) {
+        ep[qi * kEntFloats + 0] = m;
+        ep[qi * kEntFloats + 1] = s0;
+        ep[qi * kEntFloats + 2] = s1;
+      }
+    }
+}
+
+template <int D, int NT, bool ENT>
 __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
-    score_tma_kernel(Shape sh, Cache c, const bf16 *__restrict__ q, float *__restrict__ scores,
-                     float *__restrict__ tile_max, int tm_stride, int select_mode,
+    score_tma_kernel(Shape sh, Cache c, const bf16 *__restrict__ q, ScoreOut so, int select_mode,
                      const __grid_constant__ CUtensorMap kmap) {
+  float *__restrict__ scores = so.scores;
+  float *__restrict__ tile_max = so.tile_max;
+  const int tm_stride = so.tm_stride;
   using Cfg = ScoreTma<D>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t *tiles = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -228,6 +286,12 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
           v8 = fmaxf(v8, sa[nt][2 + e] + sb[nt][2 + e]);
         }
       }
+    if constexpr (ENT) {
+      const long long p0 = pbase + g, p8 = p0 + 8;
+      entropy_partials<NT>(sa, sb, p0 >= s_lo && p0 < d_lo, p8 >= s_lo && p8 < d_lo, sh.scale, sh.G,
+                           lane,
+                           so.ent + ((size_t)u * tm_stride + lt * kPartsPerTile + wg) * sh.G * kEntFloats);
+    }
     v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, 1));
     v0 = fmaxf(v0, __shfl_xor_sync(0xffffffffu, v0, 2));
     v8 = fmaxf(v8, __shfl_xor_sync(0xffffffffu, v8, 1));
@@ -251,8 +315,10 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
 
 // fp32 keys: one CTA per (tile, unit); 4 warps x 16 rows; lanes split channels.
 __global__ void __launch_bounds__(128)
-    score_f32_kernel(Shape sh, Cache c, const float *__restrict__ q, float *__restrict__ scores,
-                     float *__restrict__ tile_max, int tm_stride, int select_mode) {
+    score_f32_kernel(Shape sh, Cache c, const float *__restrict__ q, ScoreOut so, int select_mode) {
+  float *__restrict__ scores = so.scores;
+  float *__restrict__ tile_max = so.tile_max;
+  const int tm_stride = so.tm_stride;
   const int u = blockIdx.y, b = u / sh.H, h = u % sh.H;
   pdl_wait();
   pdl_launch();
@@ -268,6 +334,8 @@ __global__ void __launch_bounds__(128)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const float *kr = static_cast<const float *>(c.k_ring) + (size_t)u * sh.R * sh.d;
   float tmax = -INFINITY;
+  // raw-attention entropy partials: lane gq keeps query gq's running (m, S0, S1)
+  float em = -INFINITY, e0 = 0.f, e1 = 0.f;
   for (int r = 0; r < 16; ++r) {
     const long long pos = (long long)(ts.first + lt) * kTile + warp * 16 + r;
     if (pos < bd.s_lo || pos >= bd.d_lo) continue;
@@ -276,13 +344,32 @@ __global__ void __launch_bounds__(128)
     for (int gq = 0; gq < sh.G; ++gq) {
       float a = 0.f;
       for (int ch = lane; ch < sh.d; ch += 32) a += qs[gq * sh.d + ch] * krow[ch];
-      best = fmaxf(best, warp_sum(a));
+      a = warp_sum(a);
+      best = fmaxf(best, a);
+      if (so.ent && lane == gq) {
+        const float x = a * sh.scale;
+        if (x > em) {  // rescale the running sums to the new maximum
+          const float f = expf(em - x);
+          e1 = f * (e1 + (em - x) * e0);
+          e0 = f * e0;
+          em = x;
+        }
+        const float dd = x - em, ee = expf(dd);
+        e0 += ee;
+        e1 += ee * dd;
+      }
     }
     const float s = best * sh.scale;
     if (lane == 0) scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
     tmax = fmaxf(tmax, s);
   }
   if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + warp] = tmax;
+  if (so.ent && lane < sh.G) {
+    float *ep = so.ent + (((size_t)u * tm_stride + lt * kPartsPerTile + warp) * sh.G + lane) * kEntFloats;
+    ep[0] = em;
+    ep[1] = e0;
+    ep[2] = e1;
+  }
 }
 
 }  // namespace hardkv

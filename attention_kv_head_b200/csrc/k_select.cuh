@@ -82,6 +82,8 @@ __host__ __device__ inline size_t topp_smem_bytes(int cache_n) {
 }
 
 struct SelShared {
+  double dred[32][3];  // block reductions of the temperature solve
+  double hq[16];       // raw-attention entropy of each query of the group
   unsigned long long wmass[32];
   uint32_t wcnt[32];
   int scan[40];
@@ -233,6 +235,118 @@ __device__ __forceinline__ void warp_sort64(uint32_t (&k)[2], int (&p)[2], int l
   }
 }
 
+// Selection rule and calibration of one top-p / top-k launch.
+struct SelectParams {
+  const float *tau;   // [B,H] caller temperatures (CAL fixed), or nullptr = 1
+  const float *ent;   // raw-attention entropy partials (ScoreOut::ent): entropy-matched tau
+  float *tau_out;     // [B,H] temperature each selected unit used, or nullptr
+  float p;            // top-p mass
+  int rule;           // HARDKV_RULE_TOPP or HARDKV_RULE_TOPK
+  int k;              // RULE_TOPK: kept count (1..Cap)
+};
+
+// Sum of three doubles over the 1024-thread block; every thread gets the totals.
+__device__ __forceinline__ void block_sum3(double &a, double &b, double &c, SelShared &S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  if (lane == 0) {
+    S.dred[warp][0] = a;
+    S.dred[warp][1] = b;
+    S.dred[warp][2] = c;
+  }
+  __syncthreads();
+  a = b = c = 0.0;
+  for (int w = 0; w < kSelThreads / 32; ++w) {  // same order in every thread
+    a += S.dred[w][0];
+    b += S.dred[w][1];
+    c += S.dred[w][2];
+  }
+  __syncthreads();
+}
+
+// Merges raw-attention entropy partials (m, S0, S1) of the same query:
+// S0 = sum exp(l - m), S1 = sum exp(l - m) (l - m); m = -inf marks an empty partial.
+__device__ __forceinline__ void ent_merge(double &m, double &s0, double &s1, double pm, double p0,
+                                          double p1) {
+  if (pm == -INFINITY) return;
+  if (pm > m) {  // move the running sums to the larger reference
+    const double f = m == -INFINITY ? 0.0 : exp(m - pm);
+    s1 = f * (s1 + (m - pm) * s0);
+    s0 = f * s0;
+    m = pm;
+  }
+  const double f = exp(pm - m);
+  s1 += f * (p1 + (pm - m) * p0);
+  s0 += f * p0;
+}
+
+constexpr double kTauMin = 1.0 / 64.0, kTauMax = 64.0;  // range of the entropy-matched tau
+
+// Entropy-matched calibration temperature of unit u (the whole block calls it):
+// target = mean over the group's queries of the raw attention's entropy over the
+// candidates (from the score stage's per-part partials); tau solves
+// H(softmax(s / tau)) = target for the candidates' scores s (x = s - M <= 0).
+// H(beta = 1/tau) = ln S0 - beta S1 / S0 with S0 = sum e^(beta x), S1 = sum e^(beta x) x,
+// decreasing in beta, dH/dbeta = -beta (S2/S0 - (S1/S0)^2): Newton steps on beta kept
+// inside a shrinking bracket [1/64, 64] (a geometric bisection step whenever Newton
+// leaves it). Fewer than two candidates: tau = 1.
+__device__ float entropy_matched_tau(const Shape &sh, const SelectParams &sp, const float *src, int L,
+                                     float M, int u, int tm_stride, int nparts, SelShared &S) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (L <= 1) return 1.0f;
+  if (warp < sh.G) {  // warp g merges query g's partials over the unit's parts
+    double m = -INFINITY, s0 = 0.0, s1 = 0.0;
+    for (int i = lane; i < nparts; i += 32) {
+      const float *e = sp.ent + (((size_t)u * tm_stride + i) * sh.G + warp) * kEntFloats;
+      ent_merge(m, s0, s1, e[0], e[1], e[2]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double om = __shfl_xor_sync(0xffffffffu, m, o);
+      const double o0 = __shfl_xor_sync(0xffffffffu, s0, o);
+      const double o1 = __shfl_xor_sync(0xffffffffu, s1, o);
+      ent_merge(m, s0, s1, om, o0, o1);
+    }
+    if (lane == 0) S.hq[warp] = s0 > 0.0 ? log(s0) - s1 / s0 : 0.0;
+  }
+  __syncthreads();
+  double target = 0.0;
+  for (int g = 0; g < sh.G; ++g) target += S.hq[g];
+  target /= sh.G;
+  double lo = 1.0 / kTauMax, hi = 1.0 / kTauMin, beta = 1.0;  // bracket on beta
+  for (int it = 0; it < 64; ++it) {
+    double a = 0.0, b = 0.0, c = 0.0;
+    const float bf = (float)beta;
+    for (int j = threadIdx.x; j < L; j += kSelThreads) {
+      const float x = src[j] - M;
+      const double e = (double)expf(bf * x);
+      a += e;
+      b += e * x;
+      c += e * (double)x * x;
+    }
+    block_sum3(a, b, c, S);  // identical totals in every thread: uniform control flow
+    const double mean = b / a, h = log(a) - beta * mean;
+    const double dh = -beta * (c / a - mean * mean);
+    if (h > target)
+      lo = beta;  // entropy too high: sharpen (larger beta)
+    else
+      hi = beta;
+    double nb = dh < 0.0 ? beta - (h - target) / dh : 0.0;
+    if (!(nb > lo && nb < hi)) nb = sqrt(lo * hi);
+    if (fabs(nb - beta) <= 1e-12 * beta || hi - lo <= 1e-12 * lo) {
+      beta = nb;
+      break;
+    }
+    beta = nb;
+  }
+  return (float)(1.0 / beta);
+}
+
 // One CTA per (b,h). Writes the mask (if not NULL) and, with WRITE_IDX, the compact
 // index list sp_idx / n_kept (positions of kept candidates in ascending order).
 //
@@ -247,9 +361,12 @@ __device__ __forceinline__ void warp_sort64(uint32_t (&k)[2], int (&p)[2], int l
 // j <= pos_cut.
 template <bool WRITE_IDX>
 __global__ void __launch_bounds__(kSelThreads)
-    topp_kernel(Shape sh, Cache c, const float *__restrict__ scores,
-                const float *__restrict__ tile_max, int tm_stride, const float *__restrict__ tau,
-                float p, int select_mode, uint32_t *__restrict__ mask, int cache_n) {
+    topp_kernel(Shape sh, Cache c, ScoreOut so, SelectParams sp, int select_mode,
+                uint32_t *__restrict__ mask, int cache_n) {
+  const float *__restrict__ scores = so.scores;
+  const float *__restrict__ tile_max = so.tile_max;
+  const int tm_stride = so.tm_stride;
+  const float p = sp.p;
   const int u = blockIdx.x, b = u / sh.H;
   pdl_wait();
   pdl_launch();
@@ -269,7 +386,7 @@ __global__ void __launch_bounds__(kSelThreads)
   if (!bd.ok && tid == 0) flag(c.status, HARDKV_DEV_BAD_BOUNDS);
   const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
   const float *sc = scores + (size_t)u * sh.R;
-  const float tv = tau ? tau[u] : 1.0f;
+  float tv = sp.tau ? sp.tau[u] : 1.0f;
   const bool cached = L <= cache_n;
   const float *src = cached ? score_cache : sc;
 
@@ -300,10 +417,14 @@ __global__ void __launch_bounds__(kSelThreads)
   const float M = block_max(m, S.red);  // also publishes fill_bar's initialisation
   if (cached && L > 0 && !mbar_wait(&fill_bar, 0) && tid == 0)
     flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
+  const bool topk = sp.rule == HARDKV_RULE_TOPK;
+  if (sp.ent && !topk) tv = entropy_matched_tau(sh, sp, src, L, M, u, tm_stride, ts.n * kPartsPerTile, S);
+  if (sp.tau_out && tid == 0) sp.tau_out[u] = topk ? 1.0f : tv;
 
-  const uint32_t cap = (uint32_t)sh.cap;
-  // p >= 1 with at most Cap candidates keeps every candidate: no histogram needed
-  bool keep_all = L == 0 || (p >= 1.0f && (uint32_t)L <= cap);
+  // top-k: the k best (no mass rule); top-p: at most Cap
+  const uint32_t cap = topk ? (uint32_t)min(sp.k, sh.cap) : (uint32_t)sh.cap;
+  // p >= 1 (or top-k) with at most `cap` candidates keeps every candidate: no histogram
+  bool keep_all = L == 0 || ((topk || p >= 1.0f) && (uint32_t)L <= cap);
   // per-bin counts matter only when Cap can bind before the last candidate; otherwise
   // the count above b1 comes from the candidate pass
   const bool use_cnt = cap < (uint32_t)L;
@@ -335,8 +456,8 @@ __global__ void __launch_bounds__(kSelThreads)
     unsigned long long Z = 0;
     for (int w = 0; w < kSelThreads / 32; ++w) Z += S.wmass[w];
     __syncthreads();
-    // the threshold T = ceil(p Z) (p >= 1 keeps all, up to Cap)
-    if (p < 1.0f) T = (unsigned long long)ceil((double)p * (double)Z);
+    // the threshold T = ceil(p Z) (p >= 1 keeps all, up to Cap; top-k has no mass rule)
+    if (p < 1.0f && !topk) T = (unsigned long long)ceil((double)p * (double)Z);
   }
 
   uint32_t above_cnt = 0;
@@ -618,7 +739,7 @@ __global__ void __launch_bounds__(kSelThreads)
     if (tid == 0) c.n_kept[u] = n;
   }
   if (tid == 0) {
-    if (!keep_all && S.clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
+    if (!keep_all && !topk && S.clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
     atomicAdd(c.status + HARDKV_ST_SELECTIONS, 1u);
   }
 }

@@ -63,6 +63,19 @@ enum { HARDKV_EVICT = 0, HARDKV_MERGE = 1 };
  * MOVED = only sequences whose last hardkv_append moved a block (moved[b] != 0),
  *         i.e. each sequence reselects once per block of decode steps. */
 enum { HARDKV_SELECT_ALL = 0, HARDKV_SELECT_MOVED = 1 };
+/* Selection rule of a reselecting unit:
+ * TOPP = calibrated top-p (the method: a head-adaptive budget);
+ * TOPK = the k highest scores of every head (the fixed-budget selection the method is
+ *        compared with; sec. 2.B "Top-k vs. Top-p", sec. 4). */
+enum { HARDKV_RULE_TOPP = 0, HARDKV_RULE_TOPK = 1 };
+/* Logits Calibration temperature:
+ * TAU     = the caller's tau[b,h] (NULL: 1);
+ * ENTROPY = per (b,h), the tau in [1/64, 64] for which the entropy of softmax(s / tau)
+ *           over the candidates equals the mean entropy of the raw attention
+ *           softmax_j(q_g . k_j / sqrt(d)) of the head's queries g over the same
+ *           candidates (sec. 2.A Tier 2, a budget "based on the attention entropy";
+ *           sec. 2.B; sec. 3, distribution alterations mapped onto the raw attention). */
+enum { HARDKV_CAL_TAU = 0, HARDKV_CAL_ENTROPY = 1 };
 
 /* Device status words (caller-allocated uint32[HARDKV_STATUS_WORDS], zeroed by the
  * caller when it wants to start counting). */
@@ -126,6 +139,12 @@ typedef struct {
   float *out;               /* [B,Hq,d] attention output */
   cudaEvent_t *stage_events;/* NULL, or HARDKV_STEP_EVENTS events recorded before the
                                first stage and after each stage (capture-safe) */
+  int32_t rule;             /* HARDKV_RULE_TOPP (0, default) or HARDKV_RULE_TOPK */
+  int32_t top_k;            /* RULE_TOPK: kept count per (b,h), 1..Cap (p is ignored) */
+  int32_t calibration;      /* HARDKV_CAL_TAU (0, default) or HARDKV_CAL_ENTROPY (tau is
+                               then ignored) */
+  float *tau_out;           /* [B,H] (device) or NULL: the temperature each reselecting
+                               unit used (1 under RULE_TOPK) */
 } hardkv_step_args;
 #define HARDKV_STEP_EVENTS 6  /* start, append, condense, score, topp, attend */
 
@@ -175,6 +194,25 @@ int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cac
                                 int32_t select_mode, uint32_t *mask, void *ws,
                                 cudaStream_t stream);
 
+/* Stage 2 with the entropy-matched calibration (HARDKV_CAL_ENTROPY above): as
+ * hardkv_score_calibrate_topp, but each selected (b,h) solves its own temperature
+ * tau[b,h] in [1/64, 64] so that the calibrated distribution softmax(s / tau) over its
+ * candidates has the mean entropy of the raw attention distributions of its queries
+ * (Newton steps on 1/tau inside a bisection bracket, on the device). tau_out: device
+ * float [B,H] receiving the solved temperatures, or NULL. */
+int hardkv_score_calibrate_entropy_topp(const hardkv_desc *desc, const hardkv_cache *cache,
+                                        const void *q, float p, int32_t select_mode,
+                                        uint32_t *mask, float *tau_out, void *ws,
+                                        cudaStream_t stream);
+
+/* Stage 2 with the fixed-budget rule (HARDKV_RULE_TOPK): for each selected (b,h), the
+ * same scores s_j, then the k candidates first in the (s desc, position asc) order are
+ * kept (all of them when there are at most k); 1 <= k <= Cap. No calibration and no
+ * capacity clamp. mask as in hardkv_score_calibrate_topp. */
+int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
+                      int32_t k, int32_t select_mode, uint32_t *mask, void *ws,
+                      cudaStream_t stream);
+
 /* Stage 3 (sec. 2.C Index Regularization: Rewrite Cache + Flatten Index to the max
  * length). For each selected (b,h): the kept candidates of `mask` (device, layout as
  * above), in ascending position order, go to compact slots 0..n-1 — K and V rows
@@ -197,7 +235,8 @@ int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache,
                        const void *q, float *out, void *ws, cudaStream_t stream);
 
 /* One fused decode step (sec. 2.A four-stage pipeline): append, condense (MERGE
- * only), score + calibration + top-p, then regularize fused with attention: the
+ * only), score + calibration + selection (args->rule, args->calibration), then
+ * regularize fused with attention: the
  * kept rows are gathered once, written to the compact layout and attended in the
  * same pass. Results equal hardkv_append; hardkv_condense;
  * hardkv_score_calibrate_topp; hardkv_regularize; hardkv_decode_attn.
@@ -208,8 +247,9 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
 /* hardkv_decode_step with the per-step tensors in HOST memory (pinned memory makes
  * the copies asynchronous): args->q, k_new, v_new and tau (if not NULL) are read from
  * the host, args->out is written to the host; the copies and the step are enqueued
- * on `stream` and the caller synchronises before reading `out`. args->mask, if not
- * NULL, is a device pointer. Staging buffers live in the workspace. Pinned, mapped
+ * on `stream` and the caller synchronises before reading `out`. args->mask and
+ * args->tau_out, if not NULL, are device pointers. Every argument is checked before
+ * the first copy is enqueued. Staging buffers live in the workspace. Pinned, mapped
  * and 16-byte aligned k_new, v_new and out buffers (cudaHostAlloc memory under
  * unified addressing) are read / written by the kernels in place instead of copied;
  * q and tau are always copied. */

@@ -146,3 +146,27 @@ def test_host_entry_validates_before_any_copy(lib):
                    out.ctypes.data, None)
     assert lib.hardkv_decode_step_host(ctypes.byref(d), ctypes.byref(c), ctypes.byref(a), ws,
                                        None) == B.EINVAL
+
+
+def test_selection_rules_validate(lib):
+    """Top-k wants 1 <= k <= Cap; the fused step's rule and calibration fields are checked."""
+    d = desc()
+    c = _fake_cache()
+    ws = ctypes.c_void_p(0x7000000)
+    for k in (0, -3, d.sparse_cap + 1):
+        assert lib.hardkv_score_topk(ctypes.byref(d), ctypes.byref(c), 0x100, k, 0, 0x300, ws,
+                                     None) == B.EINVAL
+    assert lib.hardkv_score_topk(ctypes.byref(d), ctypes.byref(c), 0x100, 10, 9, 0x300, ws,
+                                 None) == B.EINVAL
+    assert lib.hardkv_score_calibrate_entropy_topp(ctypes.byref(d), ctypes.byref(c), 0x100,
+                                                   ctypes.c_float(1.5), 0, 0x300, None, ws,
+                                                   None) == B.EINVAL
+    assert lib.hardkv_score_calibrate_entropy_topp(ctypes.byref(d), ctypes.byref(c), 0x100,
+                                                   ctypes.c_float(0.9), 0, 0x300, 0x404, ws,
+                                                   None) == B.EALIGN
+    for rule, k, cal in ((2, 0, 0), (B.RULE_TOPK, 0, 0), (B.RULE_TOPK, d.sparse_cap + 1, 0),
+                         (B.RULE_TOPP, 0, 5)):
+        a = B.StepArgs(0x100, 0x200, 0x300, None, ctypes.c_float(0.9), 0, None, 0x400, None,
+                       rule, k, cal, None)
+        assert lib.hardkv_decode_step(ctypes.byref(d), ctypes.byref(c), ctypes.byref(a), ws,
+                                      None) == B.EINVAL

@@ -382,3 +382,173 @@ def test_host_entry_point_matches_device_step(pinned, with_tau):
         dc3.step(q, k, v, torch.empty_like(out), w.p, mask=mask3)
         torch.cuda.synchronize()
         assert not torch.equal(mask3, mask)
+
+
+def topk_eps(s: np.ndarray) -> float:
+    """Score rounding the top-k rule may see: the GPU's fp32 scores are within 1e-5 of
+    the fp64 ones relative to the unit's largest |s| (checked above), so two candidates
+    can swap only if their exact scores are within twice that."""
+    return 2e-5 * max(1.0, float(np.abs(s).max()) if s.size else 1.0)
+
+
+def check_selection_units(w, st, dc, mask, q_ex, k_ex, v_ex, check, units=None):
+    """Append-stepped oracle units vs the GPU mask: `check(un, qg, L, kept)` returns the
+    oracle set the GPU's kept set was accepted against (positions, local)."""
+    G = w.group
+    m = mask.cpu().numpy().view(np.uint32)
+    units = units or {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
+                      for h in range(w.n_kv_heads)}
+    for (b, h), un in units.items():
+        un.append(k_ex[b, h], v_ex[b, h])
+        L = un.d_lo - un.s_lo
+        kept = U.mask_bits(m[b, h], L)
+        check(b, h, un, q_ex[b, h * G:(h + 1) * G], L, kept)
+    return units
+
+
+@pytest.mark.parametrize("name", ["bf16_d128_g4", "f32_d64_g1", "bf16_g16", "batch5", "bf16_d64_g5"])
+@pytest.mark.parametrize("kfrac", [0.0, 0.1, 0.5, 1.0])
+def test_topk_selection_separate_and_fused(name, kfrac):
+    """Fixed-budget top-k (hardkv_score_topk and the fused step's RULE_TOPK) against the
+    oracle's top_k: the k best scores, ties to the lower position; indices bit-exact
+    except candidates whose exact score lies within the fp32 score rounding of the k-th
+    score; compaction and attention as for top-p."""
+    w = SMALL[name]
+    k_sel = max(1, int(round(kfrac * w.sparse_cap)))
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    dc2 = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    dc.append(k, v)
+    mask = dc.new_mask()
+    dc.score_topk(q, k_sel, mask)
+    mask2 = dc2.new_mask()
+    out2 = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+    dc2.step(q, k, v, out2, 1.0, mask=mask2, rule=B.RULE_TOPK, top_k=k_sel)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, mask2)
+    cmp = U.StepCompare(w.dtype)
+    n_kept = dc2.n_kept.cpu().numpy()
+    sp_idx = dc2.sp_idx.cpu().numpy()
+    o2 = out2.cpu().numpy()
+    flips = [0, 0]
+
+    def check(b, h, un, qg, L, kept):
+        s = O.score(qg, un.K[un.s_lo:un.d_lo])
+        sel = O.top_k(s, k_sel)
+        ok, nd = O.allowed_flips_topk(s, sel, kept, topk_eps(s))
+        assert ok, (name, b, h, nd)
+        flips[0] += int(nd > 0)
+        flips[1] += nd
+        assert kept.size == min(k_sel, L) == n_kept[b, h]
+        assert np.array_equal(sp_idx[b, h, :kept.size], un.s_lo + kept)
+        U.adopt_selection(un, kept)
+        cmp.attention(o2[b, h * w.group:(h + 1) * w.group], un.attend(qg), flipped=nd > 0)
+
+    check_selection_units(w, st, dc, mask, q_ex, k_ex, v_ex, check)
+    status = dc2.read_status()
+    assert status[B.ST_FLAGS] == 0 and status[B.ST_CLAMPS] == 0
+    U.record("topk", name=name, k=k_sel, flipped_units=flips[0], flipped_tokens=flips[1],
+             attention_units=cmp.units, worst_abs=cmp.worst_abs, worst_rel_l2=cmp.worst_rel)
+
+
+ENTROPY_CASES = ["bf16_d128_g4", "f32_d64_g1", "f32_d128_g4", "bf16_g16", "bf16_g8_d64", "p_low",
+                 "clamp", "batch5", "no_sparse"]
+
+
+@pytest.mark.parametrize("name", ENTROPY_CASES)
+def test_entropy_matched_calibration_separate_and_fused(name):
+    """Entropy-matched temperatures: each unit's tau (tau_out) within 1e-4 relative of the
+    oracle's bisection root of H(softmax(s/tau)) = mean_g H(raw attention of g); the mask
+    within the flip rule of the oracle's top-p at that tau (the oracle's masks at its own
+    tau are counted too); the fused step reproduces the separate call bit for bit."""
+    w = SMALL[name]
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    dc2 = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    p = synth.p_values(w)[0]
+    dc.append(k, v)
+    mask = dc.new_mask()
+    tau_out = torch.zeros(w.batch, w.n_kv_heads, dtype=torch.float32, device=dc.device)
+    dc.score_calibrate_entropy_topp(q, p, mask, tau_out=tau_out)
+    mask2 = dc2.new_mask()
+    tau2 = torch.zeros_like(tau_out)
+    out2 = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+    dc2.step(q, k, v, out2, p, mask=mask2, calibration=B.CAL_ENTROPY, tau_out=tau2)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, mask2) and torch.equal(tau_out, tau2)
+    taus = tau_out.cpu().numpy()
+    o2 = out2.cpu().numpy()
+    cmp = U.StepCompare(w.dtype)
+    stats = {"worst_tau_rel": 0.0, "masks_differing_at_oracle_tau": 0}
+
+    def check(b, h, un, qg, L, kept):
+        K = un.K[un.s_lo:un.d_lo]
+        s = O.score(qg, K)
+        tau_or = O.entropy_matched_tau(s, O.attention_entropy(qg, K))
+        tg = float(taus[b, h])
+        rel = abs(tg / tau_or - 1.0)
+        stats["worst_tau_rel"] = max(stats["worst_tau_rel"], rel)
+        assert rel <= 1e-4, (name, b, h, tg, tau_or)
+        if w.group == 1 and L > 1:
+            assert abs(tg - 1.0) <= 1e-4           # one query: the raw attention itself
+        sel = O.top_p(s, tg, p, w.sparse_cap)
+        same = cmp.selection(sel, p, kept)
+        stats["masks_differing_at_oracle_tau"] += int(
+            not np.array_equal(O.top_p(s, tau_or, p, w.sparse_cap).kept, kept))
+        U.adopt_selection(un, kept)
+        cmp.attention(o2[b, h * w.group:(h + 1) * w.group], un.attend(qg), flipped=not same)
+
+    check_selection_units(w, st, dc, mask, q_ex, k_ex, v_ex, check)
+    assert dc.read_status()[B.ST_FLAGS] == 0
+    U.record("entropy", name=name, taus=[float(x) for x in taus.reshape(-1)[:8]], **stats,
+             **cmp.summary())
+    print(name, stats, cmp.summary())
+
+
+@pytest.mark.parametrize("mode", ["topk", "entropy"])
+def test_full_size_topk_and_entropy(mode):
+    """llama8b_8k at full size, every unit: the fixed budget at the top-p run's mean kept
+    count (the same-box A/B of the pages' fixed-budget comparison), and the
+    entropy-matched calibration."""
+    w = synth.WORKLOADS["llama8b_8k"]
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+    mask = dc.new_mask()
+    tau_out = torch.zeros(w.batch, w.n_kv_heads, dtype=torch.float32, device=dc.device)
+    k_sel = 3638   # mean kept count of the calibrated top-p step (232804 / 64 units)
+    if mode == "topk":
+        dc.step(q, k, v, out, 1.0, mask=mask, rule=B.RULE_TOPK, top_k=k_sel)
+    else:
+        dc.step(q, k, v, out, w.p, mask=mask, calibration=B.CAL_ENTROPY, tau_out=tau_out)
+    torch.cuda.synchronize()
+    taus = tau_out.cpu().numpy()
+    o = out.cpu().numpy()
+    cmp = U.StepCompare(w.dtype)
+    worst = [0.0, 0]
+
+    def check(b, h, un, qg, L, kept):
+        K = un.K[un.s_lo:un.d_lo]
+        s = O.score(qg, K)
+        if mode == "topk":
+            ok, nd = O.allowed_flips_topk(s, O.top_k(s, k_sel), kept, topk_eps(s))
+            assert ok, (b, h, nd)
+            worst[1] += int(nd > 0)
+            flipped = nd > 0
+        else:
+            tau_or = O.entropy_matched_tau(s, O.attention_entropy(qg, K))
+            worst[0] = max(worst[0], abs(float(taus[b, h]) / tau_or - 1))
+            assert worst[0] <= 1e-4
+            flipped = not cmp.selection(O.top_p(s, float(taus[b, h]), w.p, w.sparse_cap), w.p, kept)
+        U.adopt_selection(un, kept)
+        cmp.attention(o[b, h * w.group:(h + 1) * w.group], un.attend(qg), flipped=flipped)
+
+    check_selection_units(w, st, dc, mask, q_ex, k_ex, v_ex, check)
+    assert dc.read_status()[B.ST_FLAGS] == 0
+    U.record("full_size_" + mode, workload=w.name, kept=int(dc.n_kept.sum()), worst_tau_rel=worst[0],
+             topk_flipped_units=worst[1], tau_min=float(taus.min()), tau_max=float(taus.max()),
+             **cmp.summary())
+    print(mode, int(dc.n_kept.sum()), worst, cmp.summary())
