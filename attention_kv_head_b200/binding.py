@@ -19,6 +19,7 @@ F32, BF16 = 0, 1
 EVICT, MERGE = 0, 1
 SELECT_ALL, SELECT_MOVED = 0, 1
 RULE_TOPP, RULE_TOPK = 0, 1
+LAYOUT_REWRITE, LAYOUT_SPARSE_LOAD, LAYOUT_MTI = 0, 1, 2
 CAL_TAU, CAL_ENTROPY = 0, 1
 STATUS_WORDS = 8
 ST_FLAGS, ST_CLAMPS, ST_NEAR_TIES, ST_MERGED, ST_MOVES, ST_SELECTIONS = range(6)
@@ -38,14 +39,19 @@ class Desc(ctypes.Structure):
 class Cache(ctypes.Structure):
     _fields_ = [(n, _vp) for n in (
         "k_ring", "v_ring", "len", "d_lo", "s_lo", "moved", "k_sp", "v_sp", "sp_idx",
-        "n_kept", "k_cd", "v_cd", "w_cd", "status")]
+        "n_kept", "sp_mode", "k_cd", "v_cd", "w_cd", "status")]
+
+
+class LayoutPolicy(ctypes.Structure):
+    _fields_ = [("mode", _i32), ("reuse_steps", _i32), ("l_lower", _i32), ("l_upper", _i32),
+                ("gather_surcharge", ctypes.c_float)]
 
 
 class StepArgs(ctypes.Structure):
     _fields_ = [("q", _vp), ("k_new", _vp), ("v_new", _vp), ("tau", _vp),
                 ("p", ctypes.c_float), ("select_mode", _i32), ("mask", _vp), ("out", _vp),
                 ("stage_events", _vp), ("rule", _i32), ("top_k", _i32), ("calibration", _i32),
-                ("tau_out", _vp)]
+                ("tau_out", _vp), ("layout", ctypes.POINTER(LayoutPolicy))]
 
 
 class HardKVError(RuntimeError):
@@ -71,6 +77,8 @@ _SIGS = {
                                          _vp, _vp, _vp]),
     "hardkv_regularize": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _i32,
                                          _vp, _vp]),
+    "hardkv_regularize_policy": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _i32,
+                                                ctypes.POINTER(LayoutPolicy), _vp, _vp]),
     "hardkv_decode_attn": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp,
                                           _vp, _vp]),
     "hardkv_decode_step": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),

@@ -49,6 +49,7 @@ class DecodeCache:
         self.v_sp = torch.zeros(Bn, H, cap, d, dtype=td, device=dev)
         self.sp_idx = torch.full((Bn, H, cap), -1, dtype=torch.int32, device=dev)
         self.n_kept = torch.zeros(Bn, H, dtype=torch.int32, device=dev)
+        self.sp_mode = torch.zeros(Bn, H, dtype=torch.int32, device=dev)
         self.k_cd = torch.zeros(Bn, H, C, d, dtype=td, device=dev)
         self.v_cd = torch.zeros(Bn, H, C, d, dtype=td, device=dev)
         self.w_cd = torch.zeros(Bn, H, C, dtype=torch.float32, device=dev)
@@ -58,7 +59,8 @@ class DecodeCache:
         self.mask_words = self.lib.hardkv_mask_words(ctypes.byref(self.desc))
         self.cstruct = B.Cache(*[_ptr(t) for t in (
             self.k_ring, self.v_ring, self.len, self.d_lo, self.s_lo, self.moved, self.k_sp,
-            self.v_sp, self.sp_idx, self.n_kept, self.k_cd, self.v_cd, self.w_cd, self.status)])
+            self.v_sp, self.sp_idx, self.n_kept, self.sp_mode, self.k_cd, self.v_cd, self.w_cd,
+            self.status)])
 
     # ------------------------------------------------------------------ state
     @classmethod
@@ -129,23 +131,28 @@ class DecodeCache:
         self._c("hardkv_score_topk", _ptr(q), int(k), select_mode, _ptr(mask), _ptr(self.ws),
                 _stream(stream))
 
-    def regularize(self, mask, select_mode=B.SELECT_ALL, stream=None):
-        self._c("hardkv_regularize", _ptr(mask), select_mode, _ptr(self.ws), _stream(stream))
+    def regularize(self, mask, select_mode=B.SELECT_ALL, stream=None, layout=None):
+        if layout is None:
+            self._c("hardkv_regularize", _ptr(mask), select_mode, _ptr(self.ws), _stream(stream))
+        else:
+            self._c("hardkv_regularize_policy", _ptr(mask), select_mode, ctypes.byref(layout),
+                    _ptr(self.ws), _stream(stream))
 
     def decode_attn(self, q, out, stream=None):
         self._c("hardkv_decode_attn", _ptr(q), _ptr(out), _ptr(self.ws), _stream(stream))
 
     def step_args(self, q, k_new, v_new, out, p, tau=None, mask=None,
                   select_mode=B.SELECT_ALL, events=None, rule=B.RULE_TOPP, top_k=0,
-                  calibration=B.CAL_TAU, tau_out=None) -> B.StepArgs:
+                  calibration=B.CAL_TAU, tau_out=None, layout=None) -> B.StepArgs:
         ev = None
         if events is not None:
             self._ev_arr = (ctypes.c_void_p * B.STEP_EVENTS)(
                 *[e.cuda_event if e is not None else None for e in events])
             ev = ctypes.cast(self._ev_arr, ctypes.c_void_p)
+        self._layout = layout          # kept alive while the call reads it
         return B.StepArgs(_ptr(q), _ptr(k_new), _ptr(v_new), _ptr(tau), ctypes.c_float(p),
                           select_mode, _ptr(mask), _ptr(out), ev, rule, int(top_k), calibration,
-                          _ptr(tau_out))
+                          _ptr(tau_out), ctypes.pointer(layout) if layout is not None else None)
 
     def step(self, q, k_new, v_new, out, p, tau=None, mask=None, select_mode=B.SELECT_ALL,
              events=None, stream=None, **sel):

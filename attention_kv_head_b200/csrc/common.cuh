@@ -25,7 +25,7 @@ struct Cache {
   void *k_ring, *v_ring;
   int32_t *len, *d_lo, *s_lo, *moved;
   void *k_sp, *v_sp;
-  int32_t *sp_idx, *n_kept;
+  int32_t *sp_idx, *n_kept, *sp_mode;
   void *k_cd, *v_cd;
   float *w_cd;
   uint32_t *status;
@@ -38,6 +38,21 @@ __device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
 // last append moved a block.
 __device__ __forceinline__ bool unit_active(int select_mode, const int32_t *moved, int b) {
   return select_mode == HARDKV_SELECT_ALL || moved[b] != 0;
+}
+
+// Layout policy as the kernels see it (reuse_steps already resolved).
+struct LayoutPolicy {
+  int mode, reuse_steps, l_lower, l_upper;
+  float gather_surcharge;
+};
+
+// Rewrite (true) or load in place (false) the n kept rows of a reselected unit.
+__device__ __forceinline__ bool layout_rewrite(const LayoutPolicy &lp, int n) {
+  if (lp.mode == HARDKV_LAYOUT_REWRITE) return true;
+  if (lp.mode == HARDKV_LAYOUT_SPARSE_LOAD) return false;
+  if (n < lp.l_lower) return false;
+  if (n > lp.l_upper) return true;
+  return 1.0 < (double)lp.reuse_steps * (double)lp.gather_surcharge;
 }
 
 __device__ __forceinline__ void flag(uint32_t *status, uint32_t bit) {

@@ -139,8 +139,9 @@ Layout layout(const hardkv_desc *d) {
 
 int check_cache(const hardkv_cache *c) {
   if (!c) return HARDKV_EINVAL;
-  const void *ptrs[] = {c->k_ring, c->v_ring, c->len, c->d_lo, c->s_lo, c->moved, c->k_sp,
-                        c->v_sp, c->sp_idx, c->n_kept, c->k_cd, c->v_cd, c->w_cd, c->status};
+  const void *ptrs[] = {c->k_ring, c->v_ring, c->len, c->d_lo,   c->s_lo, c->moved,
+                        c->k_sp,   c->v_sp,   c->sp_idx, c->n_kept, c->sp_mode, c->k_cd,
+                        c->v_cd,   c->w_cd,   c->status};
   for (const void *p : ptrs) {
     if (!p) return HARDKV_EINVAL;
     if (!aligned16(p)) return HARDKV_EALIGN;
@@ -172,6 +173,7 @@ Cache make_cache(const hardkv_cache *c) {
   k.v_sp = c->v_sp;
   k.sp_idx = c->sp_idx;
   k.n_kept = c->n_kept;
+  k.sp_mode = c->sp_mode;
   k.k_cd = c->k_cd;
   k.v_cd = c->v_cd;
   k.w_cd = c->w_cd;
@@ -420,14 +422,15 @@ int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const vo
 
 template <bool WRITE_IDX>
 int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, const SelectParams &sp,
-                int select_mode, uint32_t *mask, cudaStream_t st) {
+                int select_mode, uint32_t *mask, cudaStream_t st,
+                LayoutPolicy lp = LayoutPolicy{HARDKV_LAYOUT_REWRITE, 0, 0, 0, 0.f}) {
   const ScoreOut so = score_out(ws, L, sp.ent != nullptr);
   // the unit's scores are cached in shared memory when a whole ring fits
   const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
   const size_t smem = topp_smem_bytes(cache_n);
   HKV_TRY(set_smem(topp_kernel<WRITE_IDX>, smem));
   launch_pdl(topp_kernel<WRITE_IDX>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, so, sp,
-             select_mode, mask, cache_n);
+             select_mode, mask, cache_n, lp);
   HKV_CHECK_LAUNCH("topp_kernel");
   return HARDKV_OK;
 }
@@ -496,17 +499,40 @@ int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const v
 }
 
 int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const uint32_t *mask,
-                   int select_mode, cudaStream_t st) {
+                   int select_mode, const LayoutPolicy &lp, cudaStream_t st) {
   const dim3 grid((sh.R + kSelThreads - 1) / kSelThreads, sh.B * sh.H);
   if (d->dtype == HARDKV_BF16)
-    launch_pdl(compact_kernel<bf16>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode);
+    launch_pdl(compact_kernel<bf16>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode, lp);
   else
-    launch_pdl(compact_kernel<float>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode);
+    launch_pdl(compact_kernel<float>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode, lp);
   HKV_CHECK_LAUNCH("compact_kernel");
   return HARDKV_OK;
 }
 
 int check_p(float p) { return (p > 0.0f && p <= 1.0f) ? HARDKV_OK : HARDKV_EINVAL; }
+// Layout policy with its reuse horizon resolved for `select_mode` (NULL: rewrite).
+int layout_policy(const hardkv_desc *d, const hardkv_layout_policy *p, int select_mode,
+                  LayoutPolicy *out) {
+  LayoutPolicy lp{HARDKV_LAYOUT_REWRITE, 0, 0, 0, 0.f};
+  if (p) {
+    if (p->mode != HARDKV_LAYOUT_REWRITE && p->mode != HARDKV_LAYOUT_SPARSE_LOAD &&
+        p->mode != HARDKV_LAYOUT_MTI)
+      return HARDKV_EINVAL;
+    if (p->mode == HARDKV_LAYOUT_MTI &&
+        (p->l_lower < 0 || p->l_upper < p->l_lower || !(p->gather_surcharge >= 0.f) ||
+         !(p->gather_surcharge < 1e30f)))
+      return HARDKV_EINVAL;
+    lp.mode = p->mode;
+    lp.l_lower = p->l_lower;
+    lp.l_upper = p->l_upper;
+    lp.gather_surcharge = p->gather_surcharge;
+    lp.reuse_steps = p->reuse_steps >= 0 ? p->reuse_steps
+                                          : (select_mode == HARDKV_SELECT_MOVED ? d->block - 1 : 0);
+  }
+  *out = lp;
+  return HARDKV_OK;
+}
+
 int check_rule(const hardkv_desc *d, int rule, int k, int calibration) {
   if (rule != HARDKV_RULE_TOPP && rule != HARDKV_RULE_TOPK) return HARDKV_EINVAL;
   if (rule == HARDKV_RULE_TOPK && (k < 1 || k > d->sparse_cap)) return HARDKV_EINVAL;
@@ -625,10 +651,18 @@ int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const 
 
 int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache, const uint32_t *mask,
                       int32_t select_mode, void *ws, cudaStream_t stream) {
+  return hardkv_regularize_policy(desc, cache, mask, select_mode, nullptr, ws, stream);
+}
+
+int hardkv_regularize_policy(const hardkv_desc *desc, const hardkv_cache *cache,
+                             const uint32_t *mask, int32_t select_mode,
+                             const hardkv_layout_policy *policy, void *ws, cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_ptr(mask));
   HKV_TRY(check_mode(select_mode));
-  return launch_compact(desc, make_shape(desc), make_cache(cache), mask, select_mode, stream);
+  LayoutPolicy lp;
+  HKV_TRY(layout_policy(desc, policy, select_mode, &lp));
+  return launch_compact(desc, make_shape(desc), make_cache(cache), mask, select_mode, lp, stream);
 }
 
 int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
@@ -647,6 +681,8 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_step_args(a, false));
   HKV_TRY(check_rule(desc, a->rule, a->top_k, a->calibration));
+  LayoutPolicy lp;
+  HKV_TRY(layout_policy(desc, a->layout, a->select_mode, &lp));
   const bool entropy = a->rule == HARDKV_RULE_TOPP && a->calibration == HARDKV_CAL_ENTROPY;
   const Shape sh = make_shape(desc);
   const Cache c = make_cache(cache);
@@ -665,7 +701,7 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(record(ev, 3, stream));
   HKV_TRY(launch_topp<true>(sh, c, ws, L,
                             select_params(a->tau, a->p, a->rule, a->top_k, entropy, a->tau_out, ws, L),
-                            a->select_mode, a->mask, stream));
+                            a->select_mode, a->mask, stream, lp));
   HKV_TRY(record(ev, 4, stream));
   HKV_TRY(launch_attend(desc, sh, c, a->q, a->out, ws, L, 1, a->select_mode, false, stream));
   return record(ev, 5, stream);
@@ -691,6 +727,8 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_step_args(h, true));
   HKV_TRY(check_rule(desc, h->rule, h->top_k, h->calibration));
+  LayoutPolicy lp_check;
+  HKV_TRY(layout_policy(desc, h->layout, h->select_mode, &lp_check));
   const Layout L = layout(desc);
   const size_t e = elem_size(desc);
   const size_t U = (size_t)desc->batch * desc->n_kv_heads;

@@ -2,15 +2,17 @@
 //
 // Every unit (b,h) has a union list: [compact slots 0..n) [Dense positions d_lo..len)
 // [Condensed slots 0..C). All units' lists are concatenated and cut into contiguous
-// ranges of equal cost, one per CTA (split-K that stays balanced for ragged lengths; a
-// row gathered from the ring costs 3, any other row 2, each unit segment 320).
+// ranges of equal cost, one per CTA (split-K that stays balanced for ragged lengths;
+// the per-row and per-segment costs are kCost* below).
 // A CTA's four compute warps keep their own online-softmax states; at the end of each
 // unit segment the CTA merges them into one log-sum-exp partial, and the last CTA to
 // finish a segment of a unit (an atomic count, no waiting) merges that unit's
 // partials into the output. In fused mode the compact
 // slots of units that reselected this step are gathered from the ring (positions from
-// sp_idx) and written to the compact layout in the same pass (HARD-KV technical
-// summary sec. 2.C Rewrite Cache), so kept rows are read once.
+// sp_idx) and, for units in the Rewrite Cache layout, written to the compact layout in
+// the same pass (HARD-KV technical summary sec. 2.C Rewrite Cache), so kept rows are
+// read once; units in the Sparse Loading layout read their kept rows from the ring
+// through sp_idx at every step and are never copied.
 //
 // This file: the shared partition / row / combine code and the fp32 kernel (cp.async
 // staging, CUDA-core FMA). The bf16 kernel is in k_attend_ws.cuh.
@@ -79,17 +81,24 @@ __device__ __forceinline__ void merge_warps(const Shape &sh, const AttendParams 
 }
 
 // Partition cost of unit u: kSegCost for the segment it opens in some CTA (q load,
-// pipeline fill, partial store, count), then kCostGather per compact row gathered from
-// the ring (read, then written to its compact slot) and kCostRow per other row. The
+// pipeline fill, partial store, count), then per kept row kCostGather when it is
+// gathered from the ring and written to its compact slot (Rewrite Cache), kCostLoad when
+// it is read scattered from the ring (Sparse Loading), kCostRow per other row. The
 // weights follow measured per-row times of the bf16 kernel on B200 (about 55 ns per
 // gathered row and 37 ns per contiguous row per CTA, 6-9 us per extra segment).
-constexpr int kCostRow = 2, kCostGather = 3, kSegCost = 320;
+constexpr int kCostRow = 4, kCostLoad = 5, kCostGather = 6, kSegCost = 640;
+
+// Cost of one kept row of a unit: gather = it reselected in this (fused) launch;
+// rewrite = its selection lives in the compact layout (sp_mode).
+__device__ __forceinline__ int kept_row_cost(bool gather, bool rewrite) {
+  return rewrite ? (gather ? kCostGather : kCostRow) : kCostLoad;
+}
 
 __device__ __forceinline__ int unit_cost(const Shape &sh, const Cache &c, const AttendParams &ap, int u) {
   const int b = u / sh.H;
   const Bounds bd = load_bounds(c, b, sh.R);
   const int n = min(max(c.n_kept[u], 0), sh.cap);
-  const int wgt = (ap.fused && unit_active(ap.select_mode, c.moved, b)) ? kCostGather : kCostRow;
+  const int wgt = kept_row_cost(ap.fused && unit_active(ap.select_mode, c.moved, b), c.sp_mode[u] != 0);
   return kSegCost + (bd.ok ? wgt * n + kCostRow * (bd.len - bd.d_lo) : 0) + kCostRow * sh.C;
 }
 
@@ -245,8 +254,9 @@ constexpr uint32_t kRowGather = 1u << 29, kRowIdx = (1u << 29) - 1;
 
 struct UnitView {
   Bounds bd;
-  int n_u, nd;
-  bool gather;
+  int n_u, nd, wgt;
+  bool gather;   // reselected in this fused launch: kept rows come from the ring
+  bool rewrite;  // Rewrite Cache layout (else Sparse Loading through sp_idx)
   const int32_t *spi;
   const float *wcd;
 };
@@ -259,6 +269,8 @@ __device__ __forceinline__ UnitView unit_view(const Shape &sh, const Cache &c, c
   v.n_u = min(max(c.n_kept[u], 0), sh.cap);
   v.nd = v.bd.ok ? v.bd.len - v.bd.d_lo : 0;
   v.gather = ap.fused && unit_active(ap.select_mode, c.moved, b);
+  v.rewrite = c.sp_mode[u] != 0;
+  v.wgt = kept_row_cost(v.gather, v.rewrite);
   v.spi = c.sp_idx + (size_t)u * sh.cap;
   v.wcd = c.w_cd + (size_t)u * sh.C;
   return v;
@@ -281,11 +293,11 @@ __device__ __forceinline__ uint32_t row_decode(const Shape &sh, const UnitView &
     if (v.gather) {
       if (pos >= v.bd.s_lo && pos < v.bd.d_lo) {
         bias = 0.f;
-        return kRowRing | kRowGather | (uint32_t)(pos % sh.R);
+        return kRowRing | (v.rewrite ? kRowGather : 0u) | (uint32_t)(pos % sh.R);
       }
-    } else if (pos >= v.bd.s_lo) {
+    } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return kRowCompact | (uint32_t)j;
+      return v.rewrite ? (kRowCompact | (uint32_t)j) : (kRowRing | (uint32_t)(pos % sh.R));
     }
     return 0u;
   }
@@ -309,11 +321,11 @@ __device__ __forceinline__ uint32_t row_code(const Shape &sh, const UnitView &v,
     if (v.gather) {
       if (pos >= v.bd.s_lo && pos < v.bd.d_lo) {
         bias = 0.f;
-        return kRowRing | kRowGather | (uint32_t)(pos % sh.R);
+        return kRowRing | (v.rewrite ? kRowGather : 0u) | (uint32_t)(pos % sh.R);
       }
     } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return kRowCompact | (uint32_t)j;
+      return v.rewrite ? (kRowCompact | (uint32_t)j) : (kRowRing | (uint32_t)(pos % sh.R));
     }
     return 0u;
   }
@@ -378,9 +390,8 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
     }
     const int b = u / sh.H, h = u % sh.H;
     const UnitView v = unit_view(sh, c, ap, u);
-    const int wgt = v.gather ? kCostGather : kCostRow;
-    const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, wgt);
-    const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, wgt);
+    const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, v.wgt);
+    const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, v.wgt);
     const int ntiles = (r1 - r0 + kAttRows - 1) / kAttRows;
     const size_t rb = (size_t)D * 4;
     const uint8_t *kring = static_cast<const uint8_t *>(c.k_ring) + (size_t)u * sh.R * rb;
@@ -439,7 +450,7 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
       }
       __syncthreads();
       const uint8_t *kvb = tiles + stg * Cfg::STAGE_BYTES;
-      if (v.gather) {  // Rewrite Cache: kept rows of this tile -> compact slots
+      if (v.gather && v.rewrite) {  // Rewrite Cache: kept rows of this tile -> compact slots
         for (int i = tid; i < kAttRows * Cfg::VEC * 2; i += kF32Threads) {
           const int r = i / (2 * Cfg::VEC), kv = (i / Cfg::VEC) & 1, ch = i % Cfg::VEC;
           if (codes[stg * kAttRows + r] & kRowGather) {

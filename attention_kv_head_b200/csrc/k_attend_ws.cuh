@@ -207,9 +207,8 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
       break;
     }
     const UnitView v = unit_view(sh, c, ap, u);
-    const int wgt = v.gather ? kCostGather : kCostRow;
-    const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, wgt);
-    const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, wgt);
+    const int r0 = cost_to_row((int)(start - pre[u]), v.n_u, v.wgt);
+    const int r1 = cost_to_row((int)(min(end, (long long)pre[u + 1]) - pre[u]), v.n_u, v.wgt);
     if (r1 <= r0) {  // the range only touches this unit's segment overhead
       empty_partial(sh, ap, seg);
       if (last_to_finish(ap, pre, range, u, &s_last)) combine_unit<D>(sh, ap, pre, range, u);

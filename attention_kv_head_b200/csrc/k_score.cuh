@@ -348,7 +348,9 @@ __global__ void __launch_bounds__(128)
       best = fmaxf(best, a);
       if (so.ent && lane == gq) {
         const float x = a * sh.scale;
-        if (x > em) {  // rescale the running sums to the new maximum
+        if (em == -INFINITY) {  // first row of the part
+          em = x;
+        } else if (x > em) {  // rescale the running sums to the new maximum
           const float f = expf(em - x);
           e1 = f * (e1 + (em - x) * e0);
           e0 = f * e0;

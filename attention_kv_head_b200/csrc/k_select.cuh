@@ -274,8 +274,14 @@ __device__ __forceinline__ void block_sum3(double &a, double &b, double &c, SelS
 __device__ __forceinline__ void ent_merge(double &m, double &s0, double &s1, double pm, double p0,
                                           double p1) {
   if (pm == -INFINITY) return;
+  if (m == -INFINITY) {  // nothing merged yet (avoids -inf * 0)
+    m = pm;
+    s0 = p0;
+    s1 = p1;
+    return;
+  }
   if (pm > m) {  // move the running sums to the larger reference
-    const double f = m == -INFINITY ? 0.0 : exp(m - pm);
+    const double f = exp(m - pm);
     s1 = f * (s1 + (m - pm) * s0);
     s0 = f * s0;
     m = pm;
@@ -362,7 +368,7 @@ __device__ float entropy_matched_tau(const Shape &sh, const SelectParams &sp, co
 template <bool WRITE_IDX>
 __global__ void __launch_bounds__(kSelThreads)
     topp_kernel(Shape sh, Cache c, ScoreOut so, SelectParams sp, int select_mode,
-                uint32_t *__restrict__ mask, int cache_n) {
+                uint32_t *__restrict__ mask, int cache_n, LayoutPolicy lp) {
   const float *__restrict__ scores = so.scores;
   const float *__restrict__ tile_max = so.tile_max;
   const int tm_stride = so.tm_stride;
@@ -736,7 +742,10 @@ __global__ void __launch_bounds__(kSelThreads)
     for (int wi = nwords + tid; wi < sh.mask_words; wi += kSelThreads) mrow[wi] = 0u;
   if (WRITE_IDX) {
     for (int s2 = n + tid; s2 < sh.cap; s2 += kSelThreads) idx[s2] = -1;
-    if (tid == 0) c.n_kept[u] = n;
+    if (tid == 0) {
+      c.n_kept[u] = n;
+      c.sp_mode[u] = layout_rewrite(lp, n) ? 1 : 0;  // Rewrite Cache or Sparse Loading
+    }
   }
   if (tid == 0) {
     if (!keep_all && !topk && S.clamped) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
@@ -748,7 +757,8 @@ __global__ void __launch_bounds__(kSelThreads)
 // warp w of chunk k owns mask word 32k + w.
 template <typename T>
 __global__ void __launch_bounds__(kSelThreads)
-    compact_kernel(Shape sh, Cache c, const uint32_t *__restrict__ mask, int select_mode) {
+    compact_kernel(Shape sh, Cache c, const uint32_t *__restrict__ mask, int select_mode,
+                   LayoutPolicy lp) {
   const int u = blockIdx.y, b = u / sh.H;
   pdl_wait();
   pdl_launch();
@@ -793,11 +803,13 @@ __global__ void __launch_bounds__(kSelThreads)
   const int n_before = (int)(agg >> 32);
   const int n_total = (int)(agg & 0xffffffffull);
   const int n = min(n_total, sh.cap);
+  const bool rewrite = layout_rewrite(lp, n);  // Rewrite Cache, or the index alone
   int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
   if (chunk == 0) {
     for (int s = n + tid; s < sh.cap; s += kSelThreads) idx[s] = -1;
     if (tid == 0) {
       c.n_kept[u] = n;
+      c.sp_mode[u] = rewrite ? 1 : 0;
       if (n_total > sh.cap) atomicAdd(c.status + HARDKV_ST_CLAMPS, 1u);
     }
   }
@@ -816,6 +828,11 @@ __global__ void __launch_bounds__(kSelThreads)
   const T *vr = static_cast<const T *>(c.v_ring) + (size_t)u * sh.R * sh.d;
   T *ks = static_cast<T *>(c.k_sp) + (size_t)u * sh.cap * sh.d;
   T *vs = static_cast<T *>(c.v_sp) + (size_t)u * sh.cap * sh.d;
+  if (!rewrite) {  // Sparse Loading: the flattened index only
+    for (int e2 = tid; e2 < cnt; e2 += kSelThreads)
+      if (list_slot[e2] < sh.cap) idx[list_slot[e2]] = list_pos[e2];
+    return;
+  }
   for (int i = tid; i < cnt * 2 * vec; i += kSelThreads) {
     const int e2 = i / (2 * vec), kv = (i / vec) & 1, v2 = i % vec;
     const int slot = list_slot[e2];

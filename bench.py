@@ -167,33 +167,71 @@ def job_tokens_per_s(world: int, batch: int, max_step_ms: float) -> float:
 
 # ----------------------------------------------------------------------------- bytes
 
-def algorithmic_bytes(w, n_kept: np.ndarray, lens, d_lo, s_lo) -> dict:
-    """Bytes each stage must move (reads + writes), from the device-side kept counts."""
+def step_bytes(w, st: dict) -> dict:
+    """Bytes one decode step must move (reads + writes), per stage, from the device state
+    after the step: `st` holds len / d_lo / s_lo / moved [B], n_kept / sp_mode [B,H],
+    live [B,H] (kept rows whose position is still Sparse) and `reselect` [B] (sequences
+    that scored and selected in this step).
+
+      append    k_new, v_new read; their ring rows written
+      condense  per unit of a moved sequence (MERGE): the block's K/V and the C slots'
+                K/V read, the merged slots written back (the survey's (Blk + 2C) 2 d e)
+      score     per reselecting unit: its L candidate keys and G queries read, L fp32
+                scores written
+      topp      per reselecting unit: L scores read, the mask words and the Cap-long
+                flattened index written
+      attend    per unit: kept rows (gathered from the ring and, under Rewrite Cache,
+                written to the compact layout in a reselecting step; otherwise read from
+                the compact layout or the ring), their index, the Dense and Condensed
+                rows, the Condensed weights, q and the fp32 output"""
     e = 2 if w.dtype == "bf16" else 4
     d, H, G, C = w.head_dim, w.n_kv_heads, w.group, w.condensed_slots
-    Ls = (d_lo - s_lo).astype(np.int64)                      # per sequence
-    dense = (lens - d_lo).astype(np.int64)
+    row = 2 * d * e                                             # one K row + one V row
+    Ls = (st["d_lo"] - st["s_lo"]).astype(np.int64)            # per sequence
+    dense = (st["len"] - st["d_lo"]).astype(np.int64)
+    resel = st["reselect"].astype(bool)
+    moved = st["moved"].astype(bool)
+    n = st["n_kept"].astype(np.int64)
+    live = st["live"].astype(np.int64)
+    rw = st["sp_mode"].astype(bool)
     U = w.batch * H
-    sum_Ls = int(Ls.sum()) * H
-    sum_n = int(n_kept.sum())
-    sum_dense = int(dense.sum()) * H
-    q = w.batch * w.n_q_heads * d * e
+    q_bytes = w.batch * w.n_q_heads * d * e
+    Lsel = int(Ls[resel].sum()) * H
+    kept_sel = int(n[resel].sum())
+    gather_rw = int((n * (resel[:, None] & rw)).sum())          # gathered + written
+    gather_ld = int((n * (resel[:, None] & ~rw)).sum())         # gathered, not written
+    later = int((live * ~resel[:, None]).sum())                 # read again, either layout
     by = {
-        "append": 2 * U * d * e * 2,                                   # read k_new,v_new; write rows
-        "condense": 0,
-        "score": sum_Ls * d * e + q + sum_Ls * 4,                      # keys + q + scores
-        "topp": sum_Ls * 4 + sum_Ls // 8 + sum_n * 4,                  # scores + mask + idx
-        "attend": sum_n * 2 * d * e * 2 + sum_n * 4                    # gather read + compact write
-                  + (sum_dense + U * C) * 2 * d * e + U * C * 4 + q,  # Dense + Condensed
+        "append": 2 * U * d * e * 2,
+        "condense": (int(moved.sum()) * H * (w.block + 2 * C) * row
+                     if w.condense_mode == 1 else 0),
+        "score": Lsel * d * e + int(resel.sum()) * H * G * d * e + Lsel * 4,
+        "topp": Lsel * 4 + int(((Ls[resel] + 31) // 32).sum()) * H * 4
+                + int(resel.sum()) * H * w.sparse_cap * 4,
+        "attend": 2 * gather_rw * row + gather_ld * row + later * row + int(n.sum()) * 4
+                  + (int(dense.sum()) * H + U * C) * row + U * C * 4 + q_bytes
+                  + w.batch * w.n_q_heads * d * 4,
     }
-    by["attend"] += w.batch * w.n_q_heads * d * 4                    # output (combined in-kernel)
     by["total"] = sum(by.values())
-    by["sum_kept"] = sum_n
-    by["kept_fraction"] = sum_n / max(sum_Ls, 1)
+    by["sum_kept"] = kept_sel
+    by["kept_fraction"] = kept_sel / max(Lsel, 1)
     return by
 
 
+def sum_bytes(per_step: list) -> dict:
+    keys = ("append", "condense", "score", "topp", "attend", "total", "sum_kept")
+    out = {k: sum(b[k] for b in per_step) for k in keys}
+    sel_L = sum(b["sum_kept"] / b["kept_fraction"] for b in per_step if b["kept_fraction"] > 0)
+    out["kept_fraction"] = out["sum_kept"] / sel_L if sel_L else 0.0
+    return out
+
+
 # ----------------------------------------------------------------------------- GPU arm
+
+# Tensors of the cache state a replay starts from (the fused step changes all of them).
+STATE_TENSORS = ("len", "d_lo", "s_lo", "moved", "n_kept", "sp_mode", "sp_idx", "k_cd", "v_cd",
+                 "w_cd", "k_sp", "v_sp")
+
 
 def run_gpu(args, world, rank, local) -> dict:
     import torch
@@ -207,47 +245,105 @@ def run_gpu(args, world, rank, local) -> dict:
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = synth.WORKLOADS[args.workload].with_(seed=rank)
+    if args.p is not None:
+        w = w.with_(p=args.p)
     st = synth.initial_state(w)
     dc = DecodeCache.from_state(st, device=dev)
-    qraw, _ = synth.queries(w, 0)
-    kr, _, vr, _ = synth.step_kv(w, st.lens, 0)
-    q, k, v = dc.to_dev(qraw), dc.to_dev(kr), dc.to_dev(vr)
     p = synth.p_values(w)[0]
+    N = args.window or w.select_every                 # decode steps per timed replay
+    on_move = w.select_every > 1                      # sequences reselect on their block move
+    sel = {}
+    if args.rule == "topk":
+        k_sel = args.top_k
+        if k_sel <= 0:   # the fixed budget that keeps as many rows as calibrated top-p
+            q0, _ = synth.queries(w, 0)
+            k0, _, v0, _ = synth.step_kv(w, st.lens, 0)
+            probe = DecodeCache.from_state(st, device=dev)
+            o0 = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dev)
+            probe.step(probe.to_dev(q0), probe.to_dev(k0), probe.to_dev(v0), o0, p)
+            k_sel = max(1, int(round(float(probe.n_kept.float().mean()))))
+            del probe
+        sel.update(rule=Bn.RULE_TOPK, top_k=k_sel)
+    if args.calibration == "entropy":
+        sel.update(calibration=Bn.CAL_ENTROPY)
+    if args.layout != "rewrite":
+        sel["layout"] = Bn.LayoutPolicy(
+            Bn.LAYOUT_SPARSE_LOAD if args.layout == "sparse" else Bn.LAYOUT_MTI, -1,
+            args.l_lower, args.l_upper, args.gather_surcharge)
+    inputs = []
+    for t in range(1, N + 1) if on_move else range(N):
+        qraw, _ = synth.queries(w, t)
+        kr, _, vr, _ = synth.step_kv(w, st.lens, t)
+        inputs.append(tuple(dc.to_dev(x) for x in (qraw, kr, vr)))
     out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dev)
     mask = dc.new_mask()
-    snap = dc.snapshot_bounds()
+    mode = Bn.SELECT_MOVED if on_move else Bn.SELECT_ALL
+    stream = torch.cuda.Stream(device=dev)
+    if on_move:   # steady state: every sequence holds a selection before the window
+        q0, _ = synth.queries(w, 0)
+        k0, _, v0, _ = synth.step_kv(w, st.lens, 0)
+        with torch.cuda.stream(stream):
+            dc.step(dc.to_dev(q0), dc.to_dev(k0), dc.to_dev(v0), out, p, mask=mask, stream=stream,
+                    select_mode=Bn.SELECT_ALL, **sel)
+        stream.synchronize()
+    snap = {n_: getattr(dc, n_).clone() for n_ in STATE_TENSORS}
+
+    def restore():
+        for n_, t_ in snap.items():
+            getattr(dc, n_).copy_(t_)
+
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     def flush_l2():
         flush.zero_()                      # write 2 x L2 ...
         flush.view(torch.int32).sum()      # ... then read it back: clean lines only
-    stream = torch.cuda.Stream(device=dev)
-    evs = [torch.cuda.Event(enable_timing=True) for _ in range(Bn.STEP_EVENTS)]
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(Bn.STEP_EVENTS)] for _ in range(N)]
+
+    def window(events=False):
+        for t, (q, k, v) in enumerate(inputs):
+            dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream,
+                    events=evs[t] if events else None, **sel)
+
+    # algorithmic bytes of every step of the window, from the device state after it
+    per_step = []
     with torch.cuda.stream(stream):
-        for e_ in evs:
-            e_.record(stream)                      # create the CUDA events
+        for row in evs:
+            for e_ in row:
+                e_.record(stream)                  # create the CUDA events
+        restore()
+        for t, (q, k, v) in enumerate(inputs):
+            dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream, **sel)
+            stream.synchronize()
+            cur = {n_: getattr(dc, n_).cpu().numpy() for n_ in ("len", "d_lo", "s_lo", "moved", "n_kept",
+                                                               "sp_mode", "sp_idx")}
+            cur["reselect"] = cur["moved"] if on_move else np.ones(w.batch, bool)
+            cur["live"] = ((cur["sp_idx"] >= cur["s_lo"][:, None, None]) &
+                           (np.arange(w.sparse_cap)[None, None, :] < cur["n_kept"][:, :, None])).sum(-1)
+            per_step.append(step_bytes(w, cur))
+        by = sum_bytes(per_step)
         for _ in range(2):                         # eager warm-up (sets kernel attributes)
-            dc.restore_bounds(snap)
-            dc.step(q, k, v, out, p, mask=mask, events=evs, stream=stream)
+            restore()
+            window(events=True)
     stream.synchronize()
-    # `g` is the timed step; `gp` is the same step with event nodes between the stages
+    # `g` is the timed window; `gp` the same window with event nodes between the stages
     # (event nodes add ~2.6 us each, so they stay out of the timed graph)
     g = torch.cuda.CUDAGraph()
-    dc.restore_bounds(snap)
+    restore()
     with torch.cuda.graph(g, stream=stream):
-        dc.step(q, k, v, out, p, mask=mask)
+        window()
     gp = torch.cuda.CUDAGraph()
-    dc.restore_bounds(snap)
+    restore()
     with torch.cuda.graph(gp, stream=stream):
-        dc.step(q, k, v, out, p, mask=mask, events=evs)
+        window(events=True)
     kernels_per_step = 4 + (1 if w.condense_mode == synth.MERGE else 0)
 
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
 
-    def one_step(graph):
+    def one(graph):
         with torch.cuda.stream(stream):
-            dc.restore_bounds(snap)
+            restore()
             flush_l2()
             t0.record(stream)
             graph.replay()
@@ -256,50 +352,50 @@ def run_gpu(args, world, rank, local) -> dict:
         return t0.elapsed_time(t1)
 
     for _ in range(args.warmup):
-        one_step(g)
-        one_step(gp)
-    step_ms, stage_ms = [], []
+        one(g)
+        one(gp)
+    win_ms, stage_ms = [], []
     dist_barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clk:
         for _ in range(args.steps):
-            step_ms.append(one_step(g))
+            win_ms.append(one(g))
         for _ in range(args.steps):  # stage durations from the event-node replay
-            one_step(gp)
-            stage_ms.append([evs[i].elapsed_time(evs[i + 1]) for i in range(len(STAGES))])
+            one(gp)
+            stage_ms.append([sum(evs[t][i].elapsed_time(evs[t][i + 1]) for t in range(N))
+                             for i in range(len(STAGES))])
     torch.cuda.synchronize()
     dist_barrier(world)
-    mean_ms = float(np.mean(step_ms))
+    mean_ms = float(np.mean(win_ms)) / N              # per decode step
     max_ms = dist_max(mean_ms, world, dev)
+    stage_mean = {s: float(np.mean([x[i] for x in stage_ms])) / N for i, s in enumerate(STAGES)}
 
-    # kept counts of this step (device) -> algorithmic bytes
-    lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
-    by = algorithmic_bytes(w, dc.n_kept.cpu().numpy(), lens, dlo, slo)
-    stage_mean = {s: float(np.mean([x[i] for x in stage_ms])) for i, s in enumerate(STAGES)}
-
-    # e2e through the host-buffer entry point
-    qh, kh, vh = (t.cpu().pin_memory() for t in (q, k, v))
+    # e2e through the host-buffer entry point (every step's inputs copied in, output out)
+    host_in = [tuple(t.cpu().pin_memory() for t in x) for x in inputs]
     oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
     e2e_ms = []
     for i in range(args.warmup + args.steps):
         with torch.cuda.stream(stream):
-            dc.restore_bounds(snap)
+            restore()
             flush_l2()
-            t0 = torch.cuda.Event(enable_timing=True)
-            t1 = torch.cuda.Event(enable_timing=True)
-            t0.record(stream)
-            dc.step_host(qh, kh, vh, oh, p, mask=mask, stream=stream)
-            t1.record(stream)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for (qh, kh, vh) in host_in:
+                dc.step_host(qh, kh, vh, oh, p, mask=mask, select_mode=mode, stream=stream, **sel)
+            e1.record(stream)
         stream.synchronize()
         if i >= args.warmup:
-            e2e_ms.append(t0.elapsed_time(t1))
+            e2e_ms.append(e0.elapsed_time(e1) / N)
     e2e_mean = dist_max(float(np.mean(e2e_ms)), world, dev)
     status = dc.read_status()
+    q, k, _ = inputs[0]
     del g, gp
-    return dict(w=w, mean_ms=mean_ms, max_ms=max_ms, bytes=by, stages=stage_mean,
+    return dict(w=w, mean_ms=mean_ms, max_ms=max_ms, bytes=by, stages=stage_mean, window=N,
                 clocks=clk.summary(), e2e_ms=e2e_mean, kernels_per_step=kernels_per_step,
                 h2d=int(q.numel() * q.element_size() + 2 * k.numel() * k.element_size()),
-                d2h=int(out.numel() * 4), status=status, p50_ms=float(np.median(step_ms)))
+                d2h=int(out.numel() * 4), status=status, p50_ms=float(np.median(win_ms)) / N,
+                select=sel)
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -409,15 +505,32 @@ def main(argv=None):
     ap.add_argument("--impl", default="hardkv", choices=["hardkv", "reference"])
     ap.add_argument("--oracle-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--p", type=float, default=None, help="top-p mass (default: the workload's)")
+    ap.add_argument("--window", type=int, default=0,
+                    help="decode steps per timed replay (default: the reselection period)")
+    ap.add_argument("--rule", default="topp", choices=["topp", "topk"])
+    ap.add_argument("--top-k", type=int, default=0,
+                    help="top-k budget (0: the calibrated top-p step's mean kept count)")
+    ap.add_argument("--calibration", default="tau", choices=["tau", "entropy"])
+    ap.add_argument("--layout", default="rewrite", choices=["rewrite", "sparse", "mti"])
+    ap.add_argument("--l-lower", type=int, default=64)
+    ap.add_argument("--l-upper", type=int, default=1 << 30)
+    ap.add_argument("--gather-surcharge", type=float, default=0.5)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_info()
     from attention_kv_head_b200 import synth
     w = synth.WORKLOADS[args.workload]
+    if args.p is not None:
+        w = w.with_(p=args.p)
     config = {"workload": w.name, "batch": w.batch, "context": w.context,
-              "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim,
-              "dense_window": w.dense_window, "condensed_slots": w.condensed_slots,
-              "sparse_cap": w.sparse_cap, "p": synth.p_values(w)[0],
+              "len_range": w.len_range, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+              "head_dim": w.head_dim, "dense_window": w.dense_window,
+              "condensed_slots": w.condensed_slots, "sparse_cap": w.sparse_cap,
+              "p": synth.p_values(w)[0], "condense": "merge" if w.condense_mode else "evict",
+              "reselect": "every step" if w.select_every == 1 else "on each block move",
+              "selection": args.rule + ("" if args.rule == "topp" else f" k={args.top_k or 'auto'}"),
+              "calibration": args.calibration, "layout": args.layout,
               "l2": "flushed before every timed step: 2 x L2 written, then read back",
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -454,8 +567,12 @@ def main(argv=None):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
     r = run_gpu(args, world, rank, local)
     peaks = measured_peaks()
-    by = r["bytes"]
-    # dominant kernel by time
+    N = r["window"]
+    by = {k: (v / N if k not in ("kept_fraction",) else v) for k, v in r["bytes"].items()}
+    config["decode_steps_per_replay"] = N
+    if r["select"].get("top_k"):
+        config["selection"] = f"topk k={r['select']['top_k']}"
+    # dominant kernel by time (per decode step)
     dom = max(("score", "topp", "attend"), key=lambda s: r["stages"][s])
     dom_us = r["stages"][dom] * 1e3
     achieved = by[dom] / (dom_us * 1e-6) / 1e9
@@ -478,11 +595,13 @@ def main(argv=None):
         "step_hbm": {"alg_bytes": by["total"], "gbs": step_gbs,
                      "frac_of_8tbs": step_gbs / NOMINAL_HBM_GBS,
                      "frac_of_measured": step_gbs / peaks["hbm_gbs"],
+                     "target_frac_of_8tbs": 0.70,
+                     "meets_target": step_gbs / NOMINAL_HBM_GBS >= 0.70,
                      "kept_fraction": by["kept_fraction"], "sum_kept": by["sum_kept"],
                      "p50_ms": r["p50_ms"]},
         "stages_us": {s: round(v_ * 1e3, 2) for s, v_ in r["stages"].items()},
-        "stage_alg_bytes": {s: by[s] for s in STAGES},
-        "gpu_launches": r["kernels_per_step"] * args.steps,
+        "stage_alg_bytes": {s: int(by[s]) for s in STAGES},
+        "gpu_launches": r["kernels_per_step"] * args.steps * N,
         "clocks": r["clocks"],
         "device_status": [int(x) for x in r["status"]],
     }

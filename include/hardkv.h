@@ -76,6 +76,30 @@ enum { HARDKV_RULE_TOPP = 0, HARDKV_RULE_TOPK = 1 };
  *           candidates (sec. 2.A Tier 2, a budget "based on the attention entropy";
  *           sec. 2.B; sec. 3, distribution alterations mapped onto the raw attention). */
 enum { HARDKV_CAL_TAU = 0, HARDKV_CAL_ENTROPY = 1 };
+/* Index Regularization layout of a reselected (b,h) (sec. 2.C):
+ * REWRITE     = Rewrite Cache: the kept K/V rows are copied into the compact layout
+ *               and later steps read them there (contiguous);
+ * SPARSE_LOAD = Sparse Loading: only the flattened index (sp_idx, n_kept) is written;
+ *               attention reads the kept rows in place from the ring through it;
+ * MTI         = per (b,h), rewrite or load by the Memory-Time Integral rule of
+ *               hardkv_layout_policy. */
+enum { HARDKV_LAYOUT_REWRITE = 0, HARDKV_LAYOUT_SPARSE_LOAD = 1, HARDKV_LAYOUT_MTI = 2 };
+
+/* Layout policy of the regularization (sec. 2.C "trade-off": the one-off rewrite cost
+ * against the per-step decode gain, with budget thresholds L_lower and L_upper).
+ * Under HARDKV_LAYOUT_MTI a reselected (b,h) keeping n rows is rewritten iff
+ *   n > l_upper, or l_lower <= n <= l_upper and 1 < reuse_steps * gather_surcharge,
+ * i.e. when writing the rows once costs less than reading them scattered in each of
+ * the reuse_steps later steps that keep this selection (a contiguous read costs 1 per
+ * byte, a scattered one 1 + gather_surcharge, a write 1). */
+typedef struct {
+  int32_t mode;             /* HARDKV_LAYOUT_* */
+  int32_t reuse_steps;      /* later steps reading this selection; < 0: derived from the
+                               select mode (ALL: 0, the next step reselects; MOVED:
+                               block - 1, the selection lives until the next block move) */
+  int32_t l_lower, l_upper; /* budget thresholds (rows) */
+  float gather_surcharge;   /* > 0: extra cost per byte of a scattered row read */
+} hardkv_layout_policy;
 
 /* Device status words (caller-allocated uint32[HARDKV_STATUS_WORDS], zeroed by the
  * caller when it wants to start counting). */
@@ -122,6 +146,9 @@ typedef struct {
   void *k_sp, *v_sp;        /* [B,H,Cap,d] compact (regularized) kept rows */
   int32_t *sp_idx;          /* [B,H,Cap] position of each compact slot, -1 = pad */
   int32_t *n_kept;          /* [B,H] compact slots in use */
+  int32_t *sp_mode;         /* [B,H] layout of the unit's current selection: 1 = its rows
+                               were rewritten into k_sp / v_sp, 0 = they are loaded in
+                               place from the ring through sp_idx */
   void *k_cd, *v_cd;        /* [B,H,C,d] Condensed slots */
   float *w_cd;              /* [B,H,C] Condensed weights (tokens merged in), 0 = empty */
   uint32_t *status;         /* [HARDKV_STATUS_WORDS] device counters and flags */
@@ -145,6 +172,7 @@ typedef struct {
                                then ignored) */
   float *tau_out;           /* [B,H] (device) or NULL: the temperature each reselecting
                                unit used (1 under RULE_TOPK) */
+  const hardkv_layout_policy *layout;  /* host struct, or NULL = HARDKV_LAYOUT_REWRITE */
 } hardkv_step_args;
 #define HARDKV_STEP_EVENTS 6  /* start, append, condense, score, topp, attend */
 
@@ -223,11 +251,21 @@ int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache,
                       const uint32_t *mask, int32_t select_mode, void *ws,
                       cudaStream_t stream);
 
+/* Stage 3 with a layout policy: as hardkv_regularize, but each selected (b,h) is
+ * rewritten or only indexed (Sparse Loading) as `policy` decides (NULL = rewrite);
+ * sp_mode[b,h] records the choice for the attention of this and later steps. */
+int hardkv_regularize_policy(const hardkv_desc *desc, const hardkv_cache *cache,
+                             const uint32_t *mask, int32_t select_mode,
+                             const hardkv_layout_policy *policy, void *ws,
+                             cudaStream_t stream);
+
 /* Decode attention over the three tiers (implied by sec. 1 / sec. 5: attention runs
  * on the regularized layout). For each query head g of KV head h:
  *   out = sum_t softmax_t(l_t) v_t over
  *         Dense positions [d_lo, len)                    l = q.k / sqrt(d)
  *       U compact slots < n_kept with sp_idx >= s_lo     l = q.k / sqrt(d)
+ *         (row read from k_sp / v_sp when sp_mode = 1, from the ring row of
+ *          position sp_idx when sp_mode = 0)
  *       U Condensed slots with w > 0                     l = q.k / sqrt(d) + ln w
  * as one joint softmax (split-K partials combined by log-sum-exp).
  * out: device float [B,Hq,d]. */

@@ -552,3 +552,112 @@ def test_full_size_topk_and_entropy(mode):
              topk_flipped_units=worst[1], tau_min=float(taus.min()), tau_max=float(taus.max()),
              **cmp.summary())
     print(mode, int(dc.n_kept.sum()), worst, cmp.summary())
+
+
+def layout(mode, l_lower=0, l_upper=1 << 30, surcharge=0.5, reuse=-1):
+    return B.LayoutPolicy(mode, reuse, l_lower, l_upper, surcharge)
+
+
+@pytest.mark.parametrize("name", ["bf16_d128_g4", "f32_d64_g1", "bf16_g16", "batch5", "ring_wrap",
+                                  "clamp"])
+def test_sparse_loading_step_and_regularize(name):
+    """Sparse Loading (sec. 2.C): the fused step and hardkv_regularize_policy write the
+    same flattened index as the Rewrite Cache path but no compact rows, mark the units
+    sp_mode = 0, and the attention (which then reads the kept rows from the ring through
+    sp_idx) matches the oracle on the GPU's mask."""
+    w = SMALL[name]
+    st = synth.initial_state(w)
+    dcr, dcl, dcu = (DecodeCache.from_state(st) for _ in range(3))
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dcr, w, st, 0)
+    p = synth.p_values(w)[0]
+    mask_r, out_r = U.run_fused_step(dcr, q, k, v, p)
+    mask_l = dcl.new_mask()
+    out_l = torch.empty_like(out_r)
+    dcl.step(q, k, v, out_l, p, mask=mask_l, layout=layout(B.LAYOUT_SPARSE_LOAD))
+    # separate calls: regularize with the Sparse Loading policy, then attention
+    dcu.append(k, v)
+    mask_u = dcu.new_mask()
+    dcu.score_calibrate_topp(q, p, mask_u)
+    dcu.regularize(mask_u, layout=layout(B.LAYOUT_SPARSE_LOAD))
+    out_u = torch.empty_like(out_r)
+    dcu.decode_attn(q, out_u)
+    torch.cuda.synchronize()
+    assert torch.equal(mask_r, mask_l) and torch.equal(mask_r, mask_u)
+    for dc in (dcl, dcu):
+        assert torch.equal(dc.sp_idx, dcr.sp_idx) and torch.equal(dc.n_kept, dcr.n_kept)
+        assert int(dc.sp_mode.abs().sum()) == 0
+        assert int(dc.k_sp.abs().sum()) == 0 and int(dc.v_sp.abs().sum()) == 0   # never written
+    assert int(dcr.sp_mode.sum()) == w.units
+    cmp = U.StepCompare(w.dtype)
+    G = w.group
+    ol, ou = out_l.cpu().numpy(), out_u.cpu().numpy()
+
+    def check(b, h, un, qg, L, kept):
+        U.adopt_selection(un, kept)
+        ref = un.attend(qg)
+        cmp.attention(ol[b, h * G:(h + 1) * G], ref)
+        cmp.attention(ou[b, h * G:(h + 1) * G], ref)
+
+    check_selection_units(w, st, dcl, mask_l, q_ex, k_ex, v_ex, check)
+    U.record("sparse_load", name=name, **cmp.summary())
+
+
+@pytest.mark.parametrize("select", ["all", "moved"])
+@pytest.mark.parametrize("mode", [synth.MERGE, synth.EVICT])
+def test_multistep_mti_policy(select, mode):
+    """40 steps under the MTI policy (L_lower 96, L_upper 400, scattered-read surcharge
+    0.5): each reselecting unit's layout is the oracle's mti_rewrite decision (select on
+    move: 15 reuse steps, so budgets in [96, 400] and above are rewritten, smaller ones
+    loaded in place; select every step: nothing to reuse, everything below L_upper is
+    loaded in place); steps that do not reselect read each unit's rows from wherever its
+    layout keeps them; attention per step against the oracle."""
+    w = synth.small(condense_mode=mode, steps=40, batch=2, context=300, p=0.8,
+                    temp_range=(0.3, 6.0))
+    st = synth.initial_state(w)
+    dc = DecodeCache.from_state(st)
+    units = {(b, h): oracle_unit_from_state(st, b, h, steps=w.steps) for b in range(w.batch)
+             for h in range(w.n_kv_heads)}
+    sel_mode = B.SELECT_ALL if select == "all" else B.SELECT_MOVED
+    pol = layout(B.LAYOUT_MTI, l_lower=96, l_upper=400, surcharge=0.5)
+    cmp = U.StepCompare(w.dtype)
+    G = w.group
+    diverged, decisions = set(), {True: 0, False: 0}
+    for t in range(w.steps):
+        (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, t)
+        first = t == 0 and select == "moved"
+        mask = dc.new_mask()
+        out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+        dc.step(q, k, v, out, w.p, mask=mask, layout=pol,
+                select_mode=B.SELECT_ALL if first else sel_mode)
+        rs = "all" if first else select
+        reuse = 0 if rs == "all" else w.block - 1
+        torch.cuda.synchronize()
+        m = mask.cpu().numpy().view(np.uint32)
+        n_kept, sp_idx = dc.n_kept.cpu().numpy(), dc.sp_idx.cpu().numpy()
+        sp_mode = dc.sp_mode.cpu().numpy()
+        o = out.cpu().numpy()
+        for (b, h), un in units.items():
+            if (b, h) in diverged:
+                continue
+            res = un.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, w.p, reselect=rs)
+            if res.merge is not None and res.merge.gaps and min(res.merge.gaps) <= U.MERGE_TIE:
+                diverged.add((b, h))
+                continue
+            same, ref = True, res.out
+            if res.sel is not None:
+                L = un.d_lo - un.s_lo
+                kept = U.mask_bits(m[b, h], L)
+                same = cmp.selection(res.sel, w.p, kept)
+                if not same:
+                    U.adopt_selection(un, kept)
+                    ref = un.attend(q_ex[b, h * G:(h + 1) * G])
+                want = O.mti_rewrite(int(n_kept[b, h]), reuse, 96, 400, float(np.float32(0.5)))
+                assert bool(sp_mode[b, h]) == want, (t, b, h, int(n_kept[b, h]))
+                decisions[want] += 1
+            assert n_kept[b, h] == un.n and np.array_equal(sp_idx[b, h], un.idx)
+            cmp.attention(o[b, h * G:(h + 1) * G], ref, flipped=not same)
+    assert dc.read_status()[B.ST_FLAGS] == 0
+    if select == "moved":
+        assert decisions[True] > 0 and decisions[False] > 0      # both layouts exercised
+    U.record("multistep_mti", select=select, mode=mode, rewrite=decisions[True],
+             load=decisions[False], **cmp.summary())
