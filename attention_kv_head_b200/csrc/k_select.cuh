@@ -292,6 +292,7 @@ __device__ __forceinline__ void ent_merge(double &m, double &s0, double &s1, dou
 }
 
 constexpr double kTauMin = 1.0 / 64.0, kTauMax = 64.0;  // range of the entropy-matched tau
+constexpr int kTauIters = 48;  // bound on solver steps (a target at a range end bisects)
 
 // Entropy-matched calibration temperature of unit u (the whole block calls it):
 // target = mean over the group's queries of the raw attention's entropy over the
@@ -325,7 +326,10 @@ __device__ float entropy_matched_tau(const Shape &sh, const SelectParams &sp, co
   for (int g = 0; g < sh.G; ++g) target += S.hq[g];
   target /= sh.G;
   double lo = 1.0 / kTauMax, hi = 1.0 / kTauMin, beta = 1.0;  // bracket on beta
-  for (int it = 0; it < 64; ++it) {
+  // H(beta) is evaluated with fp32 exponentials (relative noise ~1e-7, which puts the
+  // Newton steps' floor near 1e-6 relative), so the solve stops once a step changes beta
+  // by less than 1e-5 relative; Newton needs ~5 steps
+  for (int it = 0; it < kTauIters; ++it) {
     double a = 0.0, b = 0.0, c = 0.0;
     const float bf = (float)beta;
     for (int j = threadIdx.x; j < L; j += kSelThreads) {
@@ -344,7 +348,7 @@ __device__ float entropy_matched_tau(const Shape &sh, const SelectParams &sp, co
       hi = beta;
     double nb = dh < 0.0 ? beta - (h - target) / dh : 0.0;
     if (!(nb > lo && nb < hi)) nb = sqrt(lo * hi);
-    if (fabs(nb - beta) <= 1e-12 * beta || hi - lo <= 1e-12 * lo) {
+    if (fabs(nb - beta) <= 1e-5 * beta || hi - lo <= 1e-5 * lo) {
       beta = nb;
       break;
     }
