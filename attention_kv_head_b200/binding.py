@@ -86,6 +86,7 @@ _SIGS = {
     "hardkv_decode_step_host": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),
                                                ctypes.POINTER(StepArgs), _vp, _vp]),
     "hardkv_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "hardkv_selftest_wait_timeout": (ctypes.c_int, [_vp, ctypes.c_uint32, _vp]),
     "hardkv_score_calibrate_topp_static": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache),
                                                           _vp, _vp, ctypes.c_float, _i32, _vp, _vp]),
     "hardkv_static_scratch_bytes": (ctypes.c_size_t, []),

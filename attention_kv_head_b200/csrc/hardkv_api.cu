@@ -765,6 +765,14 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   return HARDKV_OK;
 }
 
+int hardkv_selftest_wait_timeout(uint32_t *status, uint32_t limit, cudaStream_t stream) {
+  HKV_TRY(check_ptr(status));
+  if (limit < 1 || limit > (1u << 16)) return HARDKV_EINVAL;
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(status, limit);
+  HKV_CHECK_LAUNCH("wait_selftest_kernel");
+  return HARDKV_OK;
+}
+
 const char *hardkv_strerror(int code) {
   switch (code) {
     case HARDKV_OK: return "success";

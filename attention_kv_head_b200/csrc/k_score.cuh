@@ -270,6 +270,9 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
           mma_bf16(sa[nt], a, qb[nt][kk][0], qb[nt][kk][1]);
       }
     }
+    // release the stage: every lane's ldmatrix reads must be ordered before the TMA
+    // refill (a different proxy), so each lane fences before the warp's arrival
+    fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[st]);
 

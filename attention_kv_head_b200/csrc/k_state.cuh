@@ -54,6 +54,20 @@ __global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T 
   }
 }
 
+// Self-test of the bounded wait every pipeline in this library uses: one thread waits on
+// an mbarrier that nothing will ever complete, with `limit` polls. The wait must give up,
+// record HARDKV_DEV_WAIT_TIMEOUT and let the kernel return (no copy is in flight, so
+// giving up is safe here). The poll count is written to status[HARDKV_ST_FLAGS + 7].
+__global__ void wait_selftest_kernel(uint32_t *status, uint32_t limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (!mbar_wait(&bar, 0, limit)) flag(status, HARDKV_DEV_WAIT_TIMEOUT);
+  mbar_arrive(&bar);  // complete the phase so the barrier is left consistent
+  status[7] = limit;
+}
+
 __device__ __forceinline__ void store_rounded(float *p, double v) { *p = __double2float_rn(v); }
 __device__ __forceinline__ void store_rounded(bf16 *p, double v) { *p = __double2bfloat16(v); }
 

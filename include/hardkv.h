@@ -328,6 +328,14 @@ int hardkv_score_calibrate_topp_static(const hardkv_desc *desc, const hardkv_cac
 /* Size in bytes of the built-in scratch used by hardkv_score_calibrate_topp_static. */
 size_t hardkv_static_scratch_bytes(void);
 
+/* Diagnostic (no counterpart in the paper): runs the bounded wait that every pipeline
+ * of this library uses on an mbarrier that nothing completes, with at most `limit`
+ * polls (1..65536). The wait gives up, ORs HARDKV_DEV_WAIT_TIMEOUT into
+ * status[HARDKV_ST_FLAGS], writes `limit` to status[7] and the kernel returns: the
+ * path a pipeline takes when a copy never lands, exercised without any copy in flight.
+ * status: device uint32[HARDKV_STATUS_WORDS]. */
+int hardkv_selftest_wait_timeout(uint32_t *status, uint32_t limit, cudaStream_t stream);
+
 /* Human-readable text of a return code (for HARDKV_ECUDA: the last CUDA error seen
  * by this thread). The string is static or thread-local; do not free it. */
 const char *hardkv_strerror(int code);

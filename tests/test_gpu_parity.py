@@ -661,3 +661,24 @@ def test_multistep_mti_policy(select, mode):
         assert decisions[True] > 0 and decisions[False] > 0      # both layouts exercised
     U.record("multistep_mti", select=select, mode=mode, rewrite=decisions[True],
              load=decisions[False], **cmp.summary())
+
+
+def test_bounded_wait_gives_up_and_reports():
+    """The bounded mbarrier wait used by every pipeline: on a barrier nothing completes it
+    gives up after its poll limit, sets HARDKV_DEV_WAIT_TIMEOUT and the kernel returns
+    (the context stays usable: a step runs afterwards)."""
+    lib = B.load()
+    status = torch.zeros(B.STATUS_WORDS, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    assert lib.hardkv_selftest_wait_timeout(status.data_ptr(), 4096, stream) == B.OK
+    torch.cuda.synchronize()
+    st = status.cpu().numpy().view(np.uint32)
+    assert st[B.ST_FLAGS] & B.DEV_WAIT_TIMEOUT and st[7] == 4096
+    assert lib.hardkv_selftest_wait_timeout(status.data_ptr(), 0, stream) == B.EINVAL
+    w = synth.small(batch=1)
+    st0 = synth.initial_state(w)
+    dc = DecodeCache.from_state(st0)
+    (q, k, v), _ = U.upload_step(dc, w, st0, 0)
+    mask, out = U.run_fused_step(dc, q, k, v, w.p)
+    torch.cuda.synchronize()
+    assert dc.read_status()[B.ST_FLAGS] == 0 and torch.isfinite(out).all()

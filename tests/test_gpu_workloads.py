@@ -12,6 +12,7 @@ import torch
 from attention_kv_head_b200 import binding as B
 from attention_kv_head_b200 import synth
 from attention_kv_head_b200.cache import DecodeCache
+from oracle import hardkv_oracle as O
 from tests import gpu_util as U
 from tests.test_gpu_parity import oracle_unit_from_state
 
@@ -161,3 +162,38 @@ def test_stress64k_spikes_merge():
     fresh selection each step, weighted merge into 1024 slots."""
     _, n_moves = run_and_compare(synth.WORKLOADS["stress64k"], 0.95, select_on_move=False)
     assert np.all(n_moves == 7)
+
+
+@pytest.mark.parametrize("name,launches", [("long16k", 24), ("stress64k", 12)])
+def test_score_kernel_repeated_launches_full_size(name, launches):
+    """Every score of every unit, over repeated launches of the score stage at full size,
+    within 1e-5 relative of the oracle's fp64 scores. (A stage of the key pipeline reused
+    before all of its readers were done corrupts a few rows of a tile now and then; this
+    catches it where single launches and sampled units would not.)"""
+    w = synth.WORKLOADS[name]
+    st = state_of(w)
+    dc = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    dc.append(k, v)
+    torch.cuda.synchronize()
+    G, H = w.group, w.n_kv_heads
+    lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
+    K = dc.k_ring.float()
+    ref, scale = {}, {}
+    for b in range(w.batch):
+        pos = np.arange(int(slo[b]), int(dlo[b])) % st.R
+        rows = torch.from_numpy(pos).to(dc.device)
+        for h in range(H):
+            kk = K[b, h].index_select(0, rows).cpu().numpy().astype(np.float64)
+            ref[b, h] = O.score(q_ex[b, h * G:(h + 1) * G], kk)
+            scale[b, h] = max(1.0, float(np.abs(ref[b, h]).max()))
+    for t in range(launches):
+        mask = dc.new_mask()
+        dc.score_calibrate_topp(q, w.p, mask)
+        torch.cuda.synchronize()
+        sc = U.scores_from_ws(dc)
+        for (b, h), r in ref.items():
+            got = sc[b * H + h, :r.size].astype(np.float64)
+            err = np.abs(got - r).max()
+            assert err <= 1e-5 * scale[b, h], (t, b, h, err)
+    assert dc.read_status()[B.ST_FLAGS] == 0
