@@ -177,14 +177,13 @@ def test_score_kernel_repeated_launches_full_size(name, launches):
     dc.append(k, v)
     torch.cuda.synchronize()
     G, H = w.group, w.n_kv_heads
-    lens, dlo, slo = (t.cpu().numpy() for t in (dc.len, dc.d_lo, dc.s_lo))
-    K = dc.k_ring.float()
     ref, scale = {}, {}
     for b in range(w.batch):
-        pos = np.arange(int(slo[b]), int(dlo[b])) % st.R
-        rows = torch.from_numpy(pos).to(dc.device)
+        # the Sparse candidates are rows of the uploaded initial state (the append only
+        # adds a Dense row); the oracle scores them from the host arrays
+        pos = np.arange(int(st.s_lo0[b]), int(st.d_lo0[b])) % st.R
         for h in range(H):
-            kk = K[b, h].index_select(0, rows).cpu().numpy().astype(np.float64)
+            kk = U.storage_exact(st.k_ring[b, h, pos], w.dtype)
             ref[b, h] = O.score(q_ex[b, h * G:(h + 1) * G], kk)
             scale[b, h] = max(1.0, float(np.abs(ref[b, h]).max()))
     for t in range(launches):
