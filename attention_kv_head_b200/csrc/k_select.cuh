@@ -82,7 +82,9 @@ __host__ __device__ inline size_t topp_smem_bytes(int cache_n) {
 }
 
 struct SelShared {
-  double dred[32][3];  // block reductions of the temperature solve
+  double dred[32][3];  // block reductions of the temperature solve: per-warp sums
+  double dtot[3];      // and their totals (a later reduction's first barrier orders the
+                       // rewrite after every thread's read)
   double hq[16];       // raw-attention entropy of each query of the group
   unsigned long long wmass[32];
   uint32_t wcnt[32];
@@ -245,7 +247,8 @@ struct SelectParams {
   int k;              // RULE_TOPK: kept count (1..Cap)
 };
 
-// Sum of three doubles over the 1024-thread block; every thread gets the totals.
+// Sum of three doubles over the 1024-thread block; every thread gets the same totals
+// (warp sums, then warp 0 sums the 32 warp sums in a fixed shuffle order).
 __device__ __forceinline__ void block_sum3(double &a, double &b, double &c, SelShared &S) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -260,13 +263,26 @@ __device__ __forceinline__ void block_sum3(double &a, double &b, double &c, SelS
     S.dred[warp][2] = c;
   }
   __syncthreads();
-  a = b = c = 0.0;
-  for (int w = 0; w < kSelThreads / 32; ++w) {  // same order in every thread
-    a += S.dred[w][0];
-    b += S.dred[w][1];
-    c += S.dred[w][2];
+  if (warp == 0) {
+    a = S.dred[lane][0];
+    b = S.dred[lane][1];
+    c = S.dred[lane][2];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, o);
+      b += __shfl_xor_sync(0xffffffffu, b, o);
+      c += __shfl_xor_sync(0xffffffffu, c, o);
+    }
+    if (lane == 0) {
+      S.dtot[0] = a;
+      S.dtot[1] = b;
+      S.dtot[2] = c;
+    }
   }
   __syncthreads();
+  a = S.dtot[0];
+  b = S.dtot[1];
+  c = S.dtot[2];
 }
 
 // Merges raw-attention entropy partials (m, S0, S1) of the same query:

@@ -252,6 +252,7 @@ def run_gpu(args, world, rank, local) -> dict:
     p = synth.p_values(w)[0]
     N = args.window or w.select_every                 # decode steps per timed replay
     on_move = w.select_every > 1                      # sequences reselect on their block move
+    first = args.first_step if args.first_step >= 0 else (1 if on_move else 0)
     sel = {}
     if args.rule == "topk":
         k_sel = args.top_k
@@ -271,7 +272,7 @@ def run_gpu(args, world, rank, local) -> dict:
             Bn.LAYOUT_SPARSE_LOAD if args.layout == "sparse" else Bn.LAYOUT_MTI, -1,
             args.l_lower, args.l_upper, args.gather_surcharge)
     inputs = []
-    for t in range(1, N + 1) if on_move else range(N):
+    for t in range(first, first + N):
         qraw, _ = synth.queries(w, t)
         kr, _, vr, _ = synth.step_kv(w, st.lens, t)
         inputs.append(tuple(dc.to_dev(x) for x in (qraw, kr, vr)))
@@ -279,12 +280,14 @@ def run_gpu(args, world, rank, local) -> dict:
     mask = dc.new_mask()
     mode = Bn.SELECT_MOVED if on_move else Bn.SELECT_ALL
     stream = torch.cuda.Stream(device=dev)
-    if on_move:   # steady state: every sequence holds a selection before the window
-        q0, _ = synth.queries(w, 0)
-        k0, _, v0, _ = synth.step_kv(w, st.lens, 0)
+    # untimed steps before the window (the first selects every sequence, so a workload
+    # that reselects on block moves starts the window with every head holding a selection)
+    for t in range(first):
+        qs, _ = synth.queries(w, t)
+        ks, _, vs, _ = synth.step_kv(w, st.lens, t)
         with torch.cuda.stream(stream):
-            dc.step(dc.to_dev(q0), dc.to_dev(k0), dc.to_dev(v0), out, p, mask=mask, stream=stream,
-                    select_mode=Bn.SELECT_ALL, **sel)
+            dc.step(dc.to_dev(qs), dc.to_dev(ks), dc.to_dev(vs), out, p, mask=mask, stream=stream,
+                    select_mode=Bn.SELECT_ALL if t == 0 else mode, **sel)
         stream.synchronize()
     snap = {n_: getattr(dc, n_).clone() for n_ in STATE_TENSORS}
 
@@ -403,7 +406,7 @@ def run_gpu(args, world, rank, local) -> dict:
     q, k, _ = inputs[0]
     del g, gp
     return dict(w=w, mean_ms=mean_ms, max_ms=max_ms, bytes=by, stages=stage_mean, window=N,
-                outer_ms=float(np.mean(outer_ms)) / N,
+                outer_ms=float(np.mean(outer_ms)) / N, first=first,
                 clocks=clk.summary(), e2e_ms=e2e_mean, kernels_per_step=kernels_per_step,
                 h2d=int(q.numel() * q.element_size() + 2 * k.numel() * k.element_size()),
                 d2h=int(out.numel() * 4), status=status, p50_ms=float(np.median(win_ms)) / N,
@@ -520,6 +523,9 @@ def main(argv=None):
     ap.add_argument("--p", type=float, default=None, help="top-p mass (default: the workload's)")
     ap.add_argument("--window", type=int, default=0,
                     help="decode steps per timed replay (default: the reselection period)")
+    ap.add_argument("--first-step", type=int, default=-1,
+                    help="decode steps run untimed before the window (default: 1 for a "
+                         "workload that reselects on block moves, else 0)")
     ap.add_argument("--rule", default="topp", choices=["topp", "topk"])
     ap.add_argument("--top-k", type=int, default=0,
                     help="top-k budget (0: the calibrated top-p step's mean kept count)")
@@ -582,6 +588,7 @@ def main(argv=None):
     N = r["window"]
     by = {k: (v / N if k not in ("kept_fraction",) else v) for k, v in r["bytes"].items()}
     config["decode_steps_per_replay"] = N
+    config["first_timed_step"] = r["first"]
     if r["select"].get("top_k"):
         config["selection"] = f"topk k={r['select']['top_k']}"
     # dominant kernel by time (per decode step)

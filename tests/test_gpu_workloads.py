@@ -188,7 +188,7 @@ def test_score_kernel_repeated_launches_full_size(name, launches):
             scale[b, h] = max(1.0, float(np.abs(ref[b, h]).max()))
     for t in range(launches):
         mask = dc.new_mask()
-        dc.score_calibrate_topp(q, w.p, mask)
+        dc.score_calibrate_topp(q, synth.p_values(w)[0], mask)
         torch.cuda.synchronize()
         sc = U.scores_from_ws(dc)
         for (b, h), r in ref.items():
