@@ -467,9 +467,13 @@ __global__ void __launch_bounds__(kSelThreads)
       const unsigned long long mf = mass_fx(s, M, tv);
       zt += mf;
       if (use_cnt) atomicAdd(&hcnt[bin], 1u);
-      atomicAdd(&hpart[bin], (uint32_t)mf & kPartMask);
-      atomicAdd(&hpart[kBins + bin], (uint32_t)(mf >> kPartBits) & kPartMask);
-      atomicAdd(&hpart[2 * kBins + bin], (uint32_t)(mf >> (2 * kPartBits)));
+      // a part that is zero adds nothing: far below the max (mass < 2^-12, < 2^-26 of
+      // it) the upper parts vanish, so most candidates of a wide score range skip them
+      const uint32_t p0 = (uint32_t)mf & kPartMask, p1 = (uint32_t)(mf >> kPartBits) & kPartMask;
+      const uint32_t p2 = (uint32_t)(mf >> (2 * kPartBits));
+      if (p0) atomicAdd(&hpart[bin], p0);
+      if (p1) atomicAdd(&hpart[kBins + bin], p1);
+      if (p2) atomicAdd(&hpart[2 * kBins + bin], p2);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) zt += __shfl_xor_sync(0xffffffffu, zt, o);
@@ -667,15 +671,33 @@ __global__ void __launch_bounds__(kSelThreads)
           r_mass = qq < E ? (uint32_t)qq : E;
         }
         const uint32_t r = min(E, min(r_mass, cap - above_cnt));
-        // position of the r-th element with key == theta
-        int run_eq = 0;
-        for (int j0 = 0; j0 < L; j0 += kSelThreads) {
-          const int j = j0 + tid;
-          const bool eq = j < L && order_key(src[j]) == prefix;
-          const int2 e = block_scan_flag(eq, S.scan);
-          if (eq && run_eq + e.x == (int)r - 1) S.pos_cut = j;
-          run_eq += e.y;
+        // position of the r-th element (in position order) with key == theta: warp w
+        // counts the equal keys of positions [w chunk, (w+1) chunk), one prefix over the
+        // warps, then the warp holding the r-th finds it by ballots (r = 0: none kept)
+        const int chunk = ((L + 31) / 32 + kSelThreads / 32 - 1) / (kSelThreads / 32) * 32;
+        const int w0 = min(L, warp * chunk), w1 = min(L, w0 + chunk);
+        int cnt_w = 0;
+        for (int j = w0 + lane; j < w1; j += 32) cnt_w += order_key(src[j]) == prefix;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) cnt_w += __shfl_xor_sync(0xffffffffu, cnt_w, o);
+        if (tid == 0) S.pos_cut = -1;
+        if (lane == 0) S.scan[warp] = cnt_w;
+        __syncthreads();
+        int run_eq = warp_prefix_of(S.scan, warp, lane);
+        if (run_eq < (int)r && run_eq + cnt_w >= (int)r) {
+          for (int j0 = w0; j0 < w1; j0 += 32) {
+            const int j = j0 + lane;
+            const unsigned bal = __ballot_sync(0xffffffffu, j < w1 && order_key(src[j]) == prefix);
+            const int nb = __popc(bal);
+            if (run_eq + nb >= (int)r) {  // the (r - run_eq)-th set lane of this ballot
+              if (((bal >> lane) & 1u) && run_eq + __popc(bal & lt_mask) == (int)r - 1)
+                S.pos_cut = j0 + lane;
+              break;
+            }
+            run_eq += nb;
+          }
         }
+        __syncthreads();
         if (tid == 0) {
           S.theta = prefix;
           S.n_keep = (int)(above_cnt + r);
