@@ -24,6 +24,9 @@ CAL_TAU, CAL_ENTROPY = 0, 1
 STATUS_WORDS = 8
 ST_FLAGS, ST_CLAMPS, ST_NEAR_TIES, ST_MERGED, ST_MOVES, ST_SELECTIONS = range(6)
 DEV_RING_OVERFLOW, DEV_BAD_BOUNDS, DEV_SEGMENTS, DEV_WAIT_TIMEOUT = 1, 2, 4, 8
+DEV_SELECT, DEV_POOL_SHORT = 16, 32
+PAGE_ROWS = 16
+POOL_FREE, POOL_RETURNED, POOL_CTL_WORDS = 0, 1, 4
 STEP_EVENTS = 6
 
 _i32 = ctypes.c_int32
@@ -39,7 +42,8 @@ class Desc(ctypes.Structure):
 class Cache(ctypes.Structure):
     _fields_ = [(n, _vp) for n in (
         "k_ring", "v_ring", "len", "d_lo", "s_lo", "moved", "k_sp", "v_sp", "sp_idx",
-        "n_kept", "sp_mode", "k_cd", "v_cd", "w_cd", "status")]
+        "n_kept", "sp_mode", "k_cd", "v_cd", "w_cd", "status", "k_pool", "v_pool", "blk_tab",
+        "blk_cnt", "free_list", "ret_list", "pool_ctl")] + [("pool_blocks", ctypes.c_int64)]
 
 
 class LayoutPolicy(ctypes.Structure):

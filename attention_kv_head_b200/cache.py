@@ -28,7 +28,9 @@ class DecodeCache:
 
     def __init__(self, *, batch, n_q_heads, n_kv_heads, head_dim, block, dense_window,
                  condensed_slots, n_sink, sparse_cap, ring_rows, dtype, condense_mode,
-                 device="cuda"):
+                 device="cuda", pool_blocks=None):
+        """pool_blocks: None keeps Cap compact rows per head (contiguous tier); an integer
+        gives the paged tier, one pool of that many PAGE_ROWS-row blocks shared by all heads."""
         self.lib = B.load()
         self.desc = B.Desc(batch, n_q_heads, n_kv_heads, head_dim, block, dense_window,
                            condensed_slots, n_sink, sparse_cap, ring_rows,
@@ -45,8 +47,23 @@ class DecodeCache:
         self.d_lo = torch.zeros(Bn, dtype=torch.int32, device=dev)
         self.s_lo = torch.zeros(Bn, dtype=torch.int32, device=dev)
         self.moved = torch.zeros(Bn, dtype=torch.int32, device=dev)
-        self.k_sp = torch.zeros(Bn, H, cap, d, dtype=td, device=dev)
-        self.v_sp = torch.zeros(Bn, H, cap, d, dtype=td, device=dev)
+        self.pool_blocks = pool_blocks
+        if pool_blocks is None:
+            self.k_sp = torch.zeros(Bn, H, cap, d, dtype=td, device=dev)
+            self.v_sp = torch.zeros(Bn, H, cap, d, dtype=td, device=dev)
+            self.k_pool = self.v_pool = self.blk_tab = self.blk_cnt = None
+            self.free_list = self.ret_list = self.pool_ctl = None
+        else:
+            nb = int(pool_blocks)
+            tab = -(-cap // B.PAGE_ROWS)
+            self.k_sp = self.v_sp = None
+            self.k_pool = torch.zeros(nb, B.PAGE_ROWS, d, dtype=td, device=dev)
+            self.v_pool = torch.zeros(nb, B.PAGE_ROWS, d, dtype=td, device=dev)
+            self.blk_tab = torch.full((Bn, H, tab), -1, dtype=torch.int32, device=dev)
+            self.blk_cnt = torch.zeros(Bn, H, dtype=torch.int32, device=dev)
+            self.free_list = torch.arange(nb, dtype=torch.int32, device=dev)
+            self.ret_list = torch.zeros(nb, dtype=torch.int32, device=dev)
+            self.pool_ctl = torch.tensor([nb, 0, 0, 0], dtype=torch.int32, device=dev)
         self.sp_idx = torch.full((Bn, H, cap), -1, dtype=torch.int32, device=dev)
         self.n_kept = torch.zeros(Bn, H, dtype=torch.int32, device=dev)
         self.sp_mode = torch.zeros(Bn, H, dtype=torch.int32, device=dev)
@@ -60,17 +77,19 @@ class DecodeCache:
         self.cstruct = B.Cache(*[_ptr(t) for t in (
             self.k_ring, self.v_ring, self.len, self.d_lo, self.s_lo, self.moved, self.k_sp,
             self.v_sp, self.sp_idx, self.n_kept, self.sp_mode, self.k_cd, self.v_cd, self.w_cd,
-            self.status)])
+            self.status, self.k_pool, self.v_pool, self.blk_tab, self.blk_cnt, self.free_list,
+            self.ret_list, self.pool_ctl)], 0 if pool_blocks is None else int(pool_blocks))
 
     # ------------------------------------------------------------------ state
     @classmethod
-    def from_state(cls, st, device="cuda") -> "DecodeCache":
+    def from_state(cls, st, device="cuda", pool_blocks=None) -> "DecodeCache":
         """Upload a synth.InitialState."""
         w = st.w
         self = cls(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
                    head_dim=w.head_dim, block=w.block, dense_window=w.dense_window,
                    condensed_slots=w.condensed_slots, n_sink=w.n_sink, sparse_cap=w.sparse_cap,
-                   ring_rows=st.R, dtype=w.dtype, condense_mode=w.condense_mode, device=device)
+                   ring_rows=st.R, dtype=w.dtype, condense_mode=w.condense_mode, device=device,
+                   pool_blocks=pool_blocks)
         self.load_arrays(st.k_ring, st.v_ring, st.k_cd, st.v_cd, st.w_cd, st.len0, st.d_lo0,
                          st.s_lo0)
         return self

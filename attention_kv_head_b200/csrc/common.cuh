@@ -29,7 +29,22 @@ struct Cache {
   void *k_cd, *v_cd;
   float *w_cd;
   uint32_t *status;
+  // paged compact tier (k_pool == nullptr: contiguous k_sp / v_sp)
+  void *k_pool, *v_pool;
+  int32_t *blk_tab, *blk_cnt, *free_list, *ret_list, *pool_ctl;
+  int tab_blocks;  // ceil(Cap / HARDKV_PAGE_ROWS)
+  long long pool_blocks;
 };
+
+// Row (in units of d elements) of compact slot j of unit u: contiguous [U][Cap] layout,
+// or the head's block table into the pool.
+__device__ __forceinline__ size_t compact_row(const Cache &c, int cap, int u, int j) {
+  if (c.k_pool == nullptr) return (size_t)u * cap + j;
+  const int blk = c.blk_tab[(size_t)u * c.tab_blocks + j / HARDKV_PAGE_ROWS];
+  return (size_t)blk * HARDKV_PAGE_ROWS + j % HARDKV_PAGE_ROWS;
+}
+__device__ __forceinline__ void *compact_k(const Cache &c) { return c.k_pool ? c.k_pool : c.k_sp; }
+__device__ __forceinline__ void *compact_v(const Cache &c) { return c.v_pool ? c.v_pool : c.v_sp; }
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(bf16 x) { return __bfloat162float(x); }
@@ -57,6 +72,65 @@ __device__ __forceinline__ bool layout_rewrite(const LayoutPolicy &lp, int n) {
 
 __device__ __forceinline__ void flag(uint32_t *status, uint32_t bit) {
   atomicOr(status + HARDKV_ST_FLAGS, bit);
+}
+
+// Head-wise block manager (HARD-KV sec. 2.C "Metadati"). A head that needs `need` blocks
+// keeps its first min(have, need) blocks, returns the surplus to ret_list and takes the
+// deficit from the top of free_list (an atomic decrement reserves a disjoint range; a
+// range that runs below zero is short). Returned blocks join free_list only at the next
+// merge (pool_merge, run before the next allocating launch), so no block is taken and
+// returned within one launch. The calling block's thread 0 does the bookkeeping, all
+// threads copy the block ids; every thread of the block must call it. Returns the rows
+// the head's blocks hold.
+struct PoolAlloc {
+  int have, need, keep, give_at, take_from, got;
+};
+
+__device__ int pool_assign(const Cache &c, int u, int need, PoolAlloc *pa) {
+  int32_t *tab = c.blk_tab + (size_t)u * c.tab_blocks;
+  if (threadIdx.x == 0) {
+    PoolAlloc a;
+    a.have = c.blk_cnt[u];
+    a.need = need;
+    a.keep = min(a.have, need);
+    a.give_at = a.have > need ? atomicAdd(c.pool_ctl + HARDKV_POOL_RETURNED, a.have - need) : 0;
+    a.take_from = 0;
+    a.got = 0;
+    if (need > a.have) {
+      const int k = need - a.have;
+      const int t = atomicSub(c.pool_ctl + HARDKV_POOL_FREE, k);  // free count before
+      a.got = max(0, min(k, t));
+      a.take_from = t - a.got;
+      if (a.got < k) flag(c.status, HARDKV_DEV_POOL_SHORT);
+    }
+    *pa = a;
+  }
+  __syncthreads();
+  const PoolAlloc a = *pa;
+  for (int i = threadIdx.x; i < a.have - a.keep; i += blockDim.x)
+    c.ret_list[a.give_at + i] = tab[a.keep + i];
+  for (int i = threadIdx.x; i < a.got; i += blockDim.x) tab[a.keep + i] = c.free_list[a.take_from + i];
+  __syncthreads();
+  const int held = a.keep + a.got;
+  if (threadIdx.x == 0) c.blk_cnt[u] = held;
+  return held * HARDKV_PAGE_ROWS;
+}
+
+// Returned blocks join the free list (one block of threads; nothing else touches the
+// pool meanwhile: it runs before any allocating launch of a step).
+__device__ void pool_merge(const Cache &c) {
+  __shared__ int s_f, s_r;
+  if (threadIdx.x == 0) {
+    s_f = max(0, c.pool_ctl[HARDKV_POOL_FREE]);
+    s_r = c.pool_ctl[HARDKV_POOL_RETURNED];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < s_r; i += blockDim.x) c.free_list[s_f + i] = c.ret_list[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    c.pool_ctl[HARDKV_POOL_FREE] = s_f + s_r;
+    c.pool_ctl[HARDKV_POOL_RETURNED] = 0;
+  }
 }
 
 // Boundaries of sequence b, checked: 0 <= s_lo <= d_lo <= len and len - s_lo <= R.

@@ -139,13 +139,26 @@ Layout layout(const hardkv_desc *d) {
 
 int check_cache(const hardkv_cache *c) {
   if (!c) return HARDKV_EINVAL;
+  const bool paged = c->k_pool != nullptr || c->v_pool != nullptr;
   const void *ptrs[] = {c->k_ring, c->v_ring, c->len, c->d_lo,   c->s_lo, c->moved,
-                        c->k_sp,   c->v_sp,   c->sp_idx, c->n_kept, c->sp_mode, c->k_cd,
-                        c->v_cd,   c->w_cd,   c->status};
+                        c->sp_idx, c->n_kept, c->sp_mode, c->k_cd, c->v_cd, c->w_cd, c->status};
   for (const void *p : ptrs) {
     if (!p) return HARDKV_EINVAL;
     if (!aligned16(p)) return HARDKV_EALIGN;
   }
+  if (!paged) {  // contiguous compact tier
+    if (!c->k_sp || !c->v_sp) return HARDKV_EINVAL;
+    return aligned16(c->k_sp) && aligned16(c->v_sp) ? HARDKV_OK : HARDKV_EALIGN;
+  }
+  const void *pool[] = {c->k_pool, c->v_pool, c->blk_tab, c->blk_cnt, c->free_list, c->ret_list,
+                        c->pool_ctl};
+  for (const void *p : pool) {
+    if (!p) return HARDKV_EINVAL;
+    if (!aligned16(p)) return HARDKV_EALIGN;
+  }
+  // pool rows are addressed by 29-bit row codes and 32-bit block ids
+  if (c->pool_blocks < 1 || c->pool_blocks * HARDKV_PAGE_ROWS >= (int64_t(1) << 29))
+    return HARDKV_EINVAL;
   return HARDKV_OK;
 }
 
@@ -161,7 +174,7 @@ int check_common(const hardkv_desc *d, const hardkv_cache *c, const void *ws) {
   return HARDKV_OK;
 }
 
-Cache make_cache(const hardkv_cache *c) {
+Cache make_cache(const hardkv_desc *d, const hardkv_cache *c) {
   Cache k;
   k.k_ring = c->k_ring;
   k.v_ring = c->v_ring;
@@ -178,6 +191,16 @@ Cache make_cache(const hardkv_cache *c) {
   k.v_cd = c->v_cd;
   k.w_cd = c->w_cd;
   k.status = c->status;
+  const bool paged = c->k_pool != nullptr;
+  k.k_pool = paged ? c->k_pool : nullptr;
+  k.v_pool = paged ? c->v_pool : nullptr;
+  k.blk_tab = paged ? c->blk_tab : nullptr;
+  k.blk_cnt = paged ? c->blk_cnt : nullptr;
+  k.free_list = paged ? c->free_list : nullptr;
+  k.ret_list = paged ? c->ret_list : nullptr;
+  k.pool_ctl = paged ? c->pool_ctl : nullptr;
+  k.tab_blocks = (d->sparse_cap + HARDKV_PAGE_ROWS - 1) / HARDKV_PAGE_ROWS;
+  k.pool_blocks = paged ? c->pool_blocks : 0;
   return k;
 }
 
@@ -500,6 +523,12 @@ int launch_attend(const hardkv_desc *d, const Shape &sh, const Cache &c, const v
 
 int launch_compact(const hardkv_desc *d, const Shape &sh, const Cache &c, const uint32_t *mask,
                    int select_mode, const LayoutPolicy &lp, cudaStream_t st) {
+  if (c.k_pool) {  // paged tier: free the returned blocks, then size each head's blocks
+    launch_pdl(pool_merge_kernel, dim3(1), dim3(256), 0, st, c);
+    HKV_CHECK_LAUNCH("pool_merge_kernel");
+    launch_pdl(pool_alloc_kernel, dim3(sh.B * sh.H), dim3(128), 0, st, sh, c, mask, select_mode, lp);
+    HKV_CHECK_LAUNCH("pool_alloc_kernel");
+  }
   const dim3 grid((sh.R + kSelThreads - 1) / kSelThreads, sh.B * sh.H);
   if (d->dtype == HARDKV_BF16)
     launch_pdl(compact_kernel<bf16>, grid, dim3(kSelThreads), 0, st, sh, c, mask, select_mode, lp);
@@ -586,14 +615,14 @@ int hardkv_append(const hardkv_desc *desc, const hardkv_cache *cache, const void
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_ptr(k_new));
   HKV_TRY(check_ptr(v_new));
-  return launch_append(desc, make_shape(desc), make_cache(cache), k_new, v_new, ws, layout(desc),
+  return launch_append(desc, make_shape(desc), make_cache(desc, cache), k_new, v_new, ws, layout(desc),
                        stream);
 }
 
 int hardkv_condense(const hardkv_desc *desc, const hardkv_cache *cache, void *ws,
                     cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));
-  return launch_condense(desc, make_shape(desc), make_cache(cache), stream);
+  return launch_condense(desc, make_shape(desc), make_cache(desc, cache), stream);
 }
 
 int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
@@ -606,7 +635,7 @@ int hardkv_score_calibrate_topp(const hardkv_desc *desc, const hardkv_cache *cac
   HKV_TRY(check_p(p));
   HKV_TRY(check_mode(select_mode));
   const Shape sh = make_shape(desc);
-  const Cache c = make_cache(cache);
+  const Cache c = make_cache(desc, cache);
   const Layout L = layout(desc);
   HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
   return launch_topp<false>(sh, c, ws, L,
@@ -625,7 +654,7 @@ int hardkv_score_calibrate_entropy_topp(const hardkv_desc *desc, const hardkv_ca
   HKV_TRY(check_p(p));
   HKV_TRY(check_mode(select_mode));
   const Shape sh = make_shape(desc);
-  const Cache c = make_cache(cache);
+  const Cache c = make_cache(desc, cache);
   const Layout L = layout(desc);
   HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, true, stream));
   return launch_topp<false>(sh, c, ws, L,
@@ -641,7 +670,7 @@ int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const 
   HKV_TRY(check_rule(desc, HARDKV_RULE_TOPK, k, HARDKV_CAL_TAU));
   HKV_TRY(check_mode(select_mode));
   const Shape sh = make_shape(desc);
-  const Cache c = make_cache(cache);
+  const Cache c = make_cache(desc, cache);
   const Layout L = layout(desc);
   HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
   return launch_topp<false>(sh, c, ws, L,
@@ -662,7 +691,7 @@ int hardkv_regularize_policy(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(check_mode(select_mode));
   LayoutPolicy lp;
   HKV_TRY(layout_policy(desc, policy, select_mode, &lp));
-  return launch_compact(desc, make_shape(desc), make_cache(cache), mask, select_mode, lp, stream);
+  return launch_compact(desc, make_shape(desc), make_cache(desc, cache), mask, select_mode, lp, stream);
 }
 
 int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
@@ -672,7 +701,7 @@ int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const
   HKV_TRY(check_ptr(out));
   const Shape sh = make_shape(desc);
   const Layout L = layout(desc);
-  return launch_attend(desc, sh, make_cache(cache), q, out, ws, L, 0, HARDKV_SELECT_ALL, true,
+  return launch_attend(desc, sh, make_cache(desc, cache), q, out, ws, L, 0, HARDKV_SELECT_ALL, true,
                        stream);
 }
 
@@ -685,7 +714,7 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(layout_policy(desc, a->layout, a->select_mode, &lp));
   const bool entropy = a->rule == HARDKV_RULE_TOPP && a->calibration == HARDKV_CAL_ENTROPY;
   const Shape sh = make_shape(desc);
-  const Cache c = make_cache(cache);
+  const Cache c = make_cache(desc, cache);
   const Layout L = layout(desc);
   CUtensorMap kmap;
   const bool tma = desc->dtype == HARDKV_BF16;
@@ -848,7 +877,7 @@ int hardkv_score_calibrate_topp_static(const hardkv_desc *desc, const hardkv_cac
   void *ws = nullptr;
   HKV_TRY(static_scratch(&ws));
   const Shape sh = make_shape(desc);
-  const Cache c = make_cache(cache);
+  const Cache c = make_cache(desc, cache);
   HKV_TRY(launch_score(desc, sh, c, q, ws, L, select_mode, false, stream));
   return launch_topp<false>(sh, c, ws, L,
                             select_params(tau, p, HARDKV_RULE_TOPP, 0, false, nullptr, ws, L),

@@ -259,7 +259,15 @@ struct UnitView {
   bool rewrite;  // Rewrite Cache layout (else Sparse Loading through sp_idx)
   const int32_t *spi;
   const float *wcd;
+  const int32_t *tab;  // paged compact tier: this head's block table (else nullptr)
 };
+
+// Compact row of slot j: the slot itself in the head's contiguous [Cap] rows, or its
+// pool row through the head's block table (paged tier).
+__device__ __forceinline__ uint32_t compact_slot_row(const UnitView &v, int j) {
+  return v.tab ? (uint32_t)(v.tab[j / HARDKV_PAGE_ROWS] * HARDKV_PAGE_ROWS + j % HARDKV_PAGE_ROWS)
+               : (uint32_t)j;
+}
 
 __device__ __forceinline__ UnitView unit_view(const Shape &sh, const Cache &c, const AttendParams &ap,
                                               int u) {
@@ -273,6 +281,7 @@ __device__ __forceinline__ UnitView unit_view(const Shape &sh, const Cache &c, c
   v.wgt = kept_row_cost(v.gather, v.rewrite);
   v.spi = c.sp_idx + (size_t)u * sh.cap;
   v.wcd = c.w_cd + (size_t)u * sh.C;
+  v.tab = c.k_pool ? c.blk_tab + (size_t)u * c.tab_blocks : nullptr;
   return v;
 }
 
@@ -297,7 +306,7 @@ __device__ __forceinline__ uint32_t row_decode(const Shape &sh, const UnitView &
       }
     } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return v.rewrite ? (kRowCompact | (uint32_t)j) : (kRowRing | (uint32_t)(pos % sh.R));
+      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | (uint32_t)(pos % sh.R));
     }
     return 0u;
   }
@@ -325,7 +334,7 @@ __device__ __forceinline__ uint32_t row_code(const Shape &sh, const UnitView &v,
       }
     } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return v.rewrite ? (kRowCompact | (uint32_t)j) : (kRowRing | (uint32_t)(pos % sh.R));
+      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | (uint32_t)(pos % sh.R));
     }
     return 0u;
   }
@@ -396,8 +405,9 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
     const size_t rb = (size_t)D * 4;
     const uint8_t *kring = static_cast<const uint8_t *>(c.k_ring) + (size_t)u * sh.R * rb;
     const uint8_t *vring = static_cast<const uint8_t *>(c.v_ring) + (size_t)u * sh.R * rb;
-    uint8_t *ksp = static_cast<uint8_t *>(c.k_sp) + (size_t)u * sh.cap * rb;
-    uint8_t *vsp = static_cast<uint8_t *>(c.v_sp) + (size_t)u * sh.cap * rb;
+    // compact rows: the head's contiguous rows, or the pool (row codes then hold pool rows)
+    uint8_t *ksp = static_cast<uint8_t *>(compact_k(c)) + (c.k_pool ? 0 : (size_t)u * sh.cap * rb);
+    uint8_t *vsp = static_cast<uint8_t *>(compact_v(c)) + (c.k_pool ? 0 : (size_t)u * sh.cap * rb);
     const uint8_t *kcd = static_cast<const uint8_t *>(c.k_cd) + (size_t)u * sh.C * rb;
     const uint8_t *vcd = static_cast<const uint8_t *>(c.v_cd) + (size_t)u * sh.C * rb;
 
@@ -454,7 +464,7 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
         for (int i = tid; i < kAttRows * Cfg::VEC * 2; i += kF32Threads) {
           const int r = i / (2 * Cfg::VEC), kv = (i / Cfg::VEC) & 1, ch = i % Cfg::VEC;
           if (codes[stg * kAttRows + r] & kRowGather) {
-            uint8_t *dst = (kv ? vsp : ksp) + (size_t)(r0 + t * kAttRows + r) * rb + ch * 16;
+            uint8_t *dst = (kv ? vsp : ksp) + (size_t)compact_slot_row(v, r0 + t * kAttRows + r) * rb + ch * 16;
             *reinterpret_cast<uint4 *>(dst) =
                 *reinterpret_cast<const uint4 *>(kvb + kv * Cfg::TILE_BYTES + r * D * 4 + ch * 16);
           }

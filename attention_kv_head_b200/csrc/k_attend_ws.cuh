@@ -219,8 +219,9 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
     const int ntiles = (r1 - r0 + kAttRows - 1) / kAttRows;
     const uint8_t *kring = static_cast<const uint8_t *>(c.k_ring) + (size_t)u * sh.R * rb;
     const uint8_t *vring = static_cast<const uint8_t *>(c.v_ring) + (size_t)u * sh.R * rb;
-    uint8_t *ksp = static_cast<uint8_t *>(c.k_sp) + (size_t)u * sh.cap * rb;
-    uint8_t *vsp = static_cast<uint8_t *>(c.v_sp) + (size_t)u * sh.cap * rb;
+    // compact rows: the head's contiguous rows, or the pool (row codes then hold pool rows)
+    uint8_t *ksp = static_cast<uint8_t *>(compact_k(c)) + (c.k_pool ? 0 : (size_t)u * sh.cap * rb);
+    uint8_t *vsp = static_cast<uint8_t *>(compact_v(c)) + (c.k_pool ? 0 : (size_t)u * sh.cap * rb);
     const uint8_t *kcd = static_cast<const uint8_t *>(c.k_cd) + (size_t)u * sh.C * rb;
     const uint8_t *vcd = static_cast<const uint8_t *>(c.v_cd) + (size_t)u * sh.C * rb;
 
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
         const int r = k * Cfg::RPI + roff;
         const uint32_t code = __shfl_sync(0xffffffffu, cur.code, r);
         if (code & kRowGather) {
-          const size_t slot = (size_t)(r0 + t * kAttRows + w * kWsRows + r);
+          const size_t slot = compact_slot_row(v, r0 + t * kAttRows + w * kWsRows + r);
           *reinterpret_cast<uint4 *>(ksp + slot * rb + cc * 16) =
               *reinterpret_cast<const uint4 *>(ks + r * Cfg::STRIDE + cc * 16);
           *reinterpret_cast<uint4 *>(vsp + slot * rb + cc * 16) =

@@ -373,6 +373,40 @@ __device__ float entropy_matched_tau(const Shape &sh, const SelectParams &sp, co
   return (float)(1.0 / beta);
 }
 
+// ---------------------------------------------------------------- paged compact tier
+__global__ void __launch_bounds__(256) pool_merge_kernel(Cache c) {
+  pdl_wait();
+  pdl_launch();
+  pool_merge(c);
+}
+
+// Standalone regularization on the paged tier: per selected unit (one block of 128
+// threads each), the kept count of its mask and its layout decide the blocks it needs.
+__global__ void __launch_bounds__(128) pool_alloc_kernel(Shape sh, Cache c, const uint32_t *__restrict__ mask,
+                                                         int select_mode, LayoutPolicy lp) {
+  const int u = blockIdx.x, b = u / sh.H;
+  __shared__ PoolAlloc pa;
+  __shared__ int red[4];
+  pdl_wait();
+  pdl_launch();
+  if (!unit_active(select_mode, c.moved, b)) return;
+  const Bounds bd = load_bounds(c, b, sh.R);
+  const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
+  const uint32_t *mw = mask + (size_t)u * sh.mask_words;
+  int cnt = 0;
+  for (int w = threadIdx.x; w < (L + 31) / 32; w += blockDim.x) {
+    const int rem = L - 32 * w;
+    cnt += __popc(mw[w] & (rem >= 32 ? 0xffffffffu : ((1u << rem) - 1u)));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = cnt;
+  __syncthreads();
+  const int n = min(red[0] + red[1] + red[2] + red[3], sh.cap);
+  const bool rewrite = layout_rewrite(lp, n);
+  pool_assign(c, u, rewrite ? (n + HARDKV_PAGE_ROWS - 1) / HARDKV_PAGE_ROWS : 0, &pa);
+}
+
 // One CTA per (b,h). Writes the mask (if not NULL) and, with WRITE_IDX, the compact
 // index list sp_idx / n_kept (positions of kept candidates in ascending order).
 //
@@ -716,7 +750,14 @@ __global__ void __launch_bounds__(kSelThreads)
   // mask words and compact indices: warp w owns words [w K, (w+1) K), bit = lane
   const uint32_t theta = keep_all ? 0u : S.theta;
   const int pos_cut = keep_all ? 0x7fffffff : S.pos_cut;
-  const int n = keep_all ? min(L, sh.cap) : S.n_keep;
+  const int n_sel = keep_all ? min(L, sh.cap) : S.n_keep;
+  const bool rewrite = layout_rewrite(lp, n_sel);
+  int n = n_sel;  // compact slots actually written (the paged tier may hold fewer)
+  if (WRITE_IDX && c.k_pool) {
+    __shared__ PoolAlloc pa;
+    const int rows = pool_assign(c, u, rewrite ? (n_sel + HARDKV_PAGE_ROWS - 1) / HARDKV_PAGE_ROWS : 0, &pa);
+    if (rewrite) n = min(n_sel, rows);
+  }
   auto kept_at = [&](int j) -> bool {
     if (j >= L) return false;
     const uint32_t key = order_key(src[j]);
@@ -751,7 +792,7 @@ __global__ void __launch_bounds__(kSelThreads)
       for (int k = 0; k < KW; ++k) {
         const int wi = warp * K + k;
         const int slot = base + __popc(wb[k] & lt_mask);
-        if (((wb[k] >> lane) & 1u) && slot < sh.cap) idx[slot] = bd.s_lo + wi * 32 + lane;
+        if (((wb[k] >> lane) & 1u) && slot < n) idx[slot] = bd.s_lo + wi * 32 + lane;
         base += __popc(wb[k]);
       }
     }
@@ -775,7 +816,7 @@ __global__ void __launch_bounds__(kSelThreads)
         const bool kept = kept_at(j);
         const unsigned word = __ballot_sync(0xffffffffu, kept);
         const int slot = base + __popc(word & lt_mask);
-        if (kept && slot < sh.cap) idx[slot] = bd.s_lo + j;
+        if (kept && slot < n) idx[slot] = bd.s_lo + j;
         base += __popc(word);
       }
     }
@@ -786,7 +827,7 @@ __global__ void __launch_bounds__(kSelThreads)
     for (int s2 = n + tid; s2 < sh.cap; s2 += kSelThreads) idx[s2] = -1;
     if (tid == 0) {
       c.n_kept[u] = n;
-      c.sp_mode[u] = layout_rewrite(lp, n) ? 1 : 0;  // Rewrite Cache or Sparse Loading
+      c.sp_mode[u] = rewrite ? 1 : 0;  // Rewrite Cache or Sparse Loading
     }
   }
   if (tid == 0) {
@@ -844,8 +885,10 @@ __global__ void __launch_bounds__(kSelThreads)
   const unsigned long long agg = red[0];
   const int n_before = (int)(agg >> 32);
   const int n_total = (int)(agg & 0xffffffffull);
-  const int n = min(n_total, sh.cap);
-  const bool rewrite = layout_rewrite(lp, n);  // Rewrite Cache, or the index alone
+  const int n_sel = min(n_total, sh.cap);
+  const bool rewrite = layout_rewrite(lp, n_sel);  // Rewrite Cache, or the index alone
+  // the paged tier holds what pool_alloc_kernel gave the head (blk_cnt, set before)
+  const int n = (c.k_pool && rewrite) ? min(n_sel, c.blk_cnt[u] * HARDKV_PAGE_ROWS) : n_sel;
   int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
   if (chunk == 0) {
     for (int s = n + tid; s < sh.cap; s += kSelThreads) idx[s] = -1;
@@ -868,19 +911,20 @@ __global__ void __launch_bounds__(kSelThreads)
   const int vec = sh.d * (int)sizeof(T) / 16;
   const T *kr = static_cast<const T *>(c.k_ring) + (size_t)u * sh.R * sh.d;
   const T *vr = static_cast<const T *>(c.v_ring) + (size_t)u * sh.R * sh.d;
-  T *ks = static_cast<T *>(c.k_sp) + (size_t)u * sh.cap * sh.d;
-  T *vs = static_cast<T *>(c.v_sp) + (size_t)u * sh.cap * sh.d;
+  T *ks = static_cast<T *>(compact_k(c));
+  T *vs = static_cast<T *>(compact_v(c));
   if (!rewrite) {  // Sparse Loading: the flattened index only
     for (int e2 = tid; e2 < cnt; e2 += kSelThreads)
-      if (list_slot[e2] < sh.cap) idx[list_slot[e2]] = list_pos[e2];
+      if (list_slot[e2] < n) idx[list_slot[e2]] = list_pos[e2];
     return;
   }
   for (int i = tid; i < cnt * 2 * vec; i += kSelThreads) {
     const int e2 = i / (2 * vec), kv = (i / vec) & 1, v2 = i % vec;
     const int slot = list_slot[e2];
-    if (slot >= sh.cap) continue;
+    if (slot >= n) continue;
     const int pos = list_pos[e2];
-    const size_t src_row = (size_t)(pos % sh.R) * sh.d, dst_row = (size_t)slot * sh.d;
+    const size_t src_row = (size_t)(pos % sh.R) * sh.d,
+                 dst_row = compact_row(c, sh.cap, u, slot) * sh.d;
     if (kv == 0) {
       reinterpret_cast<uint4 *>(ks + dst_row)[v2] = reinterpret_cast<const uint4 *>(kr + src_row)[v2];
       if (v2 == 0) idx[slot] = pos;

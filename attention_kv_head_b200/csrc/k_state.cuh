@@ -14,6 +14,7 @@ __global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T 
   const int b = blockIdx.x;
   pdl_wait();  // the previous step's kernels finish before this one touches the state
   pdl_launch();
+  if (b == 0 && c.k_pool) pool_merge(c);  // blocks returned last step become free
   // attention completion counters of this sequence's units start the step at zero
   if (counters)
     for (int h = threadIdx.x; h < sh.H; h += blockDim.x) counters[b * sh.H + h] = 0;

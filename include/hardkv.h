@@ -117,6 +117,13 @@ enum {
 #define HARDKV_DEV_SEGMENTS      4u  /* attention partition had to drop a segment */
 #define HARDKV_DEV_WAIT_TIMEOUT  8u  /* a pipeline wait hit its iteration limit */
 #define HARDKV_DEV_SELECT       16u  /* top-p found no cut (inconsistent input): unit kept all */
+#define HARDKV_DEV_POOL_SHORT   32u  /* paged compact tier: a rewritten selection got fewer
+                                        blocks than it needed and kept its first rows only */
+
+/* Rows per block of the paged compact tier (hardkv_cache::k_pool). */
+#define HARDKV_PAGE_ROWS 16
+/* Words of hardkv_cache::pool_ctl. */
+enum { HARDKV_POOL_FREE = 0, HARDKV_POOL_RETURNED = 1, HARDKV_POOL_CTL_WORDS = 4 };
 
 /* Static shape of one attention layer's cascade cache. */
 typedef struct {
@@ -152,6 +159,30 @@ typedef struct {
   void *k_cd, *v_cd;        /* [B,H,C,d] Condensed slots */
   float *w_cd;              /* [B,H,C] Condensed weights (tokens merged in), 0 = empty */
   uint32_t *status;         /* [HARDKV_STATUS_WORDS] device counters and flags */
+  /* Paged compact tier: the head-wise block manager (sec. 2.C "Metadati": fine-grained,
+   * head-adaptive allocation with static shapes and persistent pointers). k_pool NULL:
+   * compact rows live in k_sp / v_sp ([B,H,Cap,d], Cap rows reserved per head). Otherwise
+   * k_sp / v_sp are unused (may be NULL) and compact slot j of (b,h) is row
+   *   blk_tab[(b*H + h) * tab_blocks + j / HARDKV_PAGE_ROWS] * HARDKV_PAGE_ROWS
+   *     + j % HARDKV_PAGE_ROWS
+   * of k_pool / v_pool, with tab_blocks = ceil(Cap / HARDKV_PAGE_ROWS): each head holds
+   * only the blocks its current selection needs, from one pool shared by all heads.
+   * A head that reselects with the Rewrite Cache layout and keeps n rows ends with
+   * ceil(n / HARDKV_PAGE_ROWS) blocks (a Sparse-Loading head with none): it keeps its
+   * first blocks, returns the rest to ret_list and takes what it lacks from the top of
+   * free_list. Returned blocks join free_list at the start of the next step (in the
+   * append kernel, or before a standalone regularization). If free_list runs short the
+   * head keeps the rows its blocks hold, in position order, and HARDKV_DEV_POOL_SHORT
+   * is raised. The caller sets up free_list = {0, 1, ..., pool_blocks-1},
+   * pool_ctl = {pool_blocks, 0, 0, 0} and blk_cnt = 0 once; everything after that is
+   * kept on the device. */
+  void *k_pool, *v_pool;    /* [pool_blocks, HARDKV_PAGE_ROWS, d] or NULL */
+  int32_t *blk_tab;         /* [B, H, tab_blocks] block ids of each head's compact slots */
+  int32_t *blk_cnt;         /* [B, H] blocks each head holds */
+  int32_t *free_list;       /* [pool_blocks] free block ids, [0, pool_ctl[FREE]) valid */
+  int32_t *ret_list;        /* [pool_blocks] block ids returned since the last merge */
+  int32_t *pool_ctl;        /* [HARDKV_POOL_CTL_WORDS] free count, returned count */
+  int64_t pool_blocks;      /* blocks in the pool (ignored when k_pool is NULL) */
 } hardkv_cache;
 
 /* Arguments of one fused decode step. */

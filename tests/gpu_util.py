@@ -48,6 +48,22 @@ def oracle_unit(w: synth.Workload, st: synth.InitialState, b: int, h: int, steps
                   int(st.s_lo0[b]), L0 + steps + 1)
 
 
+def oracle_unit_from_state(st: synth.InitialState, b: int, h: int, steps: int = 1):
+    """Oracle unit built from the very host arrays uploaded to the GPU."""
+    w = st.w
+    C, R = w.condensed_slots, st.R
+    L0 = int(st.len0[b])
+    K = np.zeros((L0, w.head_dim))
+    V = np.zeros((L0, w.head_dim))
+    K[:C] = storage_exact(st.k_cd[b, h], w.dtype)
+    V[:C] = storage_exact(st.v_cd[b, h], w.dtype)
+    pos = np.arange(C, L0)
+    K[C:] = storage_exact(st.k_ring[b, h, pos % R], w.dtype)
+    V[C:] = storage_exact(st.v_ring[b, h, pos % R], w.dtype)
+    return O.Unit(oracle_params(w), K, V, K[:C], V[:C], st.w_cd[b, h].astype(np.float64), L0,
+                  int(st.d_lo0[b]), int(st.s_lo0[b]), L0 + steps + 1)
+
+
 def mask_bits(mask_words_row: np.ndarray, L: int) -> np.ndarray:
     """Local indices j < L whose bit is set in one unit's mask words."""
     words = mask_words_row.astype(np.uint32)

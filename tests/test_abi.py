@@ -74,10 +74,19 @@ def test_merge_slot_limit(lib):
     assert lib.hardkv_validate(ctypes.byref(desc(condense_mode=B.MERGE, condensed_slots=4096))) == B.EINVAL
 
 
-def _fake_cache(misalign=None, null=None):
+POOL_FIELDS = ("k_pool", "v_pool", "blk_tab", "blk_cnt", "free_list", "ret_list", "pool_ctl")
+
+
+def _fake_cache(misalign=None, null=None, paged=False):
     vals = {}
     for i, (name, _) in enumerate(B.Cache._fields_):
         vals[name] = 0x10000 * (i + 1)
+    if not paged:  # contiguous compact tier: the pool fields stay NULL
+        for name in POOL_FIELDS:
+            vals[name] = None
+        vals["pool_blocks"] = 0
+    else:
+        vals["pool_blocks"] = 4096
     if misalign:
         vals[misalign] += 4
     if null:
@@ -111,6 +120,32 @@ def test_entry_points_validate_before_any_launch(lib):
     assert lib.hardkv_decode_step(ctypes.byref(d), ctypes.byref(c), ctypes.byref(args), ws,
                                   None) == B.EINVAL
     assert lib.hardkv_decode_step_host(ctypes.byref(d), ctypes.byref(c), None, ws, None) == B.EINVAL
+
+
+def test_paged_cache_validates(lib):
+    """The paged compact tier: k_sp / v_sp may be NULL, every pool pointer is required and
+    aligned, and the pool must be addressable by the 29-bit row codes."""
+    d = desc()
+    ws = ctypes.c_void_p(0x7000000)
+
+    def append(c, k_new=0x100):
+        return lib.hardkv_append(ctypes.byref(d), ctypes.byref(c), k_new, 0x200, ws, None)
+
+    # a valid paged cache gets past the cache check: the misaligned k_new decides
+    c = _fake_cache(paged=True)
+    c.k_sp = c.v_sp = None
+    assert append(c, k_new=0x104) == B.EALIGN
+    assert append(_fake_cache(null="k_sp")) == B.EINVAL  # contiguous tier needs k_sp
+    for name in POOL_FIELDS:
+        assert append(_fake_cache(paged=True, null=name)) == B.EINVAL, name
+        assert append(_fake_cache(paged=True, misalign=name)) == B.EALIGN, name
+    for blocks in (0, -1, (1 << 29) // B.PAGE_ROWS):
+        c = _fake_cache(paged=True)
+        c.pool_blocks = blocks
+        assert append(c) == B.EINVAL, blocks
+    c = _fake_cache(paged=True)
+    c.pool_blocks = (1 << 29) // B.PAGE_ROWS - 1
+    assert append(c, k_new=0x104) == B.EALIGN
 
 
 def test_strerror(lib):
