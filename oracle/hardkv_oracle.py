@@ -20,6 +20,8 @@ every formula below is a stated reading, listed in the repository's design notes
              mass >= p (p >= 1 keeps all); clamp to the capacity  (sec. 2.A Tier 2)
   regularize kept rows in ascending position order, idx = position,
              index padded with -1 to the capacity                 (sec. 2.C Rewrite / Flatten)
+  flatten    the heads' index lists end to end, offsets = exclusive running sum of
+  (sum form) the kept counts                                       (sec. 2.C Flatten to the sum)
   condense   oldest Sparse block -> EVICT (drop) or MERGE: each token, in position
              order, into the non-sink slot of highest cosine similarity (ties -> lowest
              slot); k,v <- (w k + x)/(w+1) computed in float64, rounded to the
@@ -311,6 +313,20 @@ def regularize(mask: np.ndarray, positions: np.ndarray, k_rows: np.ndarray,
     idx = np.full(cap, -1, np.int64)
     idx[:n] = positions[sel]
     return n, idx, k_rows[sel], v_rows[sel]
+
+
+def flatten_sum(index_lists):
+    """Flatten Index to the sum of the lengths (sec. 2.C: indices are regularized either
+    to the maximum length -- `regularize`'s padded [Cap] rows -- or to their sum). The
+    heads' kept-position lists are laid end to end in head order (b major, then h);
+    offsets[u] counts the entries before head u, offsets[U] all of them."""
+    offsets = [0]
+    flat = []
+    for lst in index_lists:
+        for pos in lst:
+            flat.append(int(pos))
+        offsets.append(offsets[-1] + len(lst))
+    return np.array(offsets, np.int64), np.array(flat, np.int64)
 
 
 # ----------------------------------------------------------------------------

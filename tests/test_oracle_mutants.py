@@ -122,6 +122,26 @@ def _mti_le(n, reuse_steps, l_lower, l_upper, gather_surcharge, write_cost=1.0):
     return write_cost <= reuse_steps * gather_surcharge
 
 
+def _flatten_sum_inclusive(index_lists):
+    # offsets[u] counts head u's own entries too (an inclusive running sum)
+    offsets, flat, run = [], [], 0
+    for lst in index_lists:
+        run += len(lst)
+        offsets.append(run)
+        flat.extend(int(x) for x in lst)
+    offsets.append(run)
+    return np.array(offsets, np.int64), np.array(flat, np.int64)
+
+
+def _flatten_sum_reversed_heads(index_lists):
+    lists = list(index_lists)[::-1]
+    offsets, flat = [0], []
+    for lst in lists:
+        flat.extend(int(x) for x in lst)
+        offsets.append(offsets[-1] + len(lst))
+    return np.array(offsets, np.int64), np.array(flat, np.int64)
+
+
 _orig_top_k = O.top_k
 
 MUTANTS = [
@@ -149,6 +169,9 @@ MUTANTS = [
     ("top_k", _top_k_position_desc, [lambda: [P.test_top_k_brute_force_small(s) for s in range(20)]]),
     ("top_k", _top_k_one_more, [lambda: [P.test_top_k_brute_force_small(s) for s in range(20)]]),
     ("mti_rewrite", _mti_le, [P.test_mti_policy_thresholds_and_break_even]),
+    ("flatten_sum", _flatten_sum_inclusive, [P.test_flatten_sum_hand_cases]),
+    ("flatten_sum", _flatten_sum_reversed_heads,
+     [P.test_flatten_sum_hand_cases, P.test_flatten_sum_round_trips_the_max_length_form]),
 ]
 
 

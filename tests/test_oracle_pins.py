@@ -238,6 +238,33 @@ def test_regularize_truncates_to_capacity_in_position_order():
     assert n == 20 and idx[:20].tolist() == list(range(20)) and kc.shape == (20, 50)
 
 
+def test_flatten_sum_hand_cases():
+    for c in GOLD["flatten_sum"]:
+        offsets, flat = O.flatten_sum([np.array(x, np.int64) for x in c["lists"]])
+        assert offsets.tolist() == c["offsets"], c["why"]
+        assert flat.tolist() == c["flat"], c["why"]
+
+
+def test_flatten_sum_round_trips_the_max_length_form():
+    """The sum form holds exactly the max-length form's non-pad entries: slicing the flat
+    list by the offsets gives back each head's regularized index, and the total is the
+    sum of the kept counts."""
+    r = rng(31)
+    cap, rows, ns = 40, [], []
+    for u in range(9):
+        mask = r.random(60) < r.random()
+        n, idx, _, _ = O.regularize(mask, np.arange(100 * u, 100 * u + 60), np.zeros((60, 1)),
+                                    np.zeros((60, 1)), cap)
+        rows.append(idx)
+        ns.append(n)
+    offsets, flat = O.flatten_sum([row[:n] for row, n in zip(rows, ns)])
+    assert offsets[0] == 0 and offsets[-1] == sum(ns) == flat.size
+    assert np.all(np.diff(offsets) == np.array(ns))
+    for u, (row, n) in enumerate(zip(rows, ns)):
+        seg = flat[offsets[u]:offsets[u + 1]]
+        assert np.array_equal(seg, row[:n]) and np.all(row[n:] == -1)
+
+
 # ---------------------------------------------------------------- merge / condense
 
 def test_merge_hand_case():
