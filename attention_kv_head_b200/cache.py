@@ -157,6 +157,18 @@ class DecodeCache:
             self._c("hardkv_regularize_policy", _ptr(mask), select_mode, ctypes.byref(layout),
                     _ptr(self.ws), _stream(stream))
 
+    def flatten_sum(self, offsets=None, flat=None, stream=None):
+        """Sum form of the flattened index: (offsets [B*H+1], flat [B*H*Cap]) int32;
+        flat[offsets[u]:offsets[u+1]] is unit u's kept positions."""
+        d = self.desc
+        U = d.batch * d.n_kv_heads
+        if offsets is None:
+            offsets = torch.empty(U + 1, dtype=torch.int32, device=self.device)
+        if flat is None:
+            flat = torch.empty(U * d.sparse_cap, dtype=torch.int32, device=self.device)
+        self._c("hardkv_flatten_sum", _ptr(offsets), _ptr(flat), _stream(stream))
+        return offsets, flat
+
     def decode_attn(self, q, out, stream=None):
         self._c("hardkv_decode_attn", _ptr(q), _ptr(out), _ptr(self.ws), _stream(stream))
 

@@ -694,6 +694,20 @@ int hardkv_regularize_policy(const hardkv_desc *desc, const hardkv_cache *cache,
   return launch_compact(desc, make_shape(desc), make_cache(desc, cache), mask, select_mode, lp, stream);
 }
 
+int hardkv_flatten_sum(const hardkv_desc *desc, const hardkv_cache *cache, int32_t *offsets,
+                       int32_t *flat, cudaStream_t stream) {
+  HKV_TRY(validate_desc(desc));
+  HKV_TRY(check_cache(cache));
+  HKV_TRY(check_ptr(offsets));
+  HKV_TRY(check_ptr(flat));
+  // validate_desc keeps B*H*Cap below 2^31, so every offset fits an int32
+  const Shape sh = make_shape(desc);
+  launch_pdl(flatten_sum_kernel, dim3(sh.B * sh.H), dim3(256), 0, stream, sh, make_cache(desc, cache),
+             offsets, flat);
+  HKV_CHECK_LAUNCH("flatten_sum_kernel");
+  return HARDKV_OK;
+}
+
 int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const void *q,
                        float *out, void *ws, cudaStream_t stream) {
   HKV_TRY(check_common(desc, cache, ws));

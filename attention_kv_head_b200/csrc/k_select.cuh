@@ -934,4 +934,34 @@ __global__ void __launch_bounds__(kSelThreads)
   }
 }
 
+// Flatten Index to the sum of the lengths (sec. 2.C): one CTA per unit u writes
+// offsets[u] = sum of the kept counts of the units before it (offsets[U] = the total,
+// by the last unit) and copies its n_kept index entries to flat[offsets[u] ...). The
+// running sum is re-summed per CTA (U^2 / threads reads of n_kept, all in L2), which
+// keeps it one launch with no inter-CTA ordering.
+__global__ void __launch_bounds__(256) flatten_sum_kernel(Shape sh, Cache c, int32_t *offsets,
+                                                          int32_t *flat) {
+  const int u = blockIdx.x, U = gridDim.x, tid = threadIdx.x;
+  __shared__ int red[8];
+  pdl_wait();
+  pdl_launch();
+  auto kept = [&](int v) { return min(max(c.n_kept[v], 0), sh.cap); };
+  int s = 0;
+  for (int v = tid; v < u; v += 256) s += kept(v);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if ((tid & 31) == 0) red[tid >> 5] = s;
+  __syncthreads();
+  int base = 0;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) base += red[w];
+  const int n = kept(u);
+  if (tid == 0) {
+    offsets[u] = base;
+    if (u == U - 1) offsets[U] = base + n;
+  }
+  const int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
+  for (int j = tid; j < n; j += 256) flat[base + j] = idx[j];
+}
+
 }  // namespace hardkv

@@ -290,6 +290,18 @@ int hardkv_regularize_policy(const hardkv_desc *desc, const hardkv_cache *cache,
                              const hardkv_layout_policy *policy, void *ws,
                              cudaStream_t stream);
 
+/* Flatten Index to the sum of the lengths (sec. 2.C: the index is regularized to the
+ * maximum length -- sp_idx [B,H,Cap], padded with -1 -- or to the sum of the lengths).
+ * Reads n_kept and sp_idx of every (b,h) (u = b*H + h) and writes, on the device,
+ *   offsets[u] = sum_{v < u} n_kept[v],   offsets[B*H] = sum of all n_kept,
+ *   flat[offsets[u] + j] = sp_idx[u, j]   for j < n_kept[u]
+ * (n_kept clamped to [0, Cap]). offsets: int32 [B*H + 1]; flat: int32 with room for
+ * B*H*Cap entries (the largest total); both 16-byte aligned, owned by the caller.
+ * Entries of flat past the total are not written (a valid descriptor keeps B*H*Cap
+ * below 2^31, so the offsets fit an int32). */
+int hardkv_flatten_sum(const hardkv_desc *desc, const hardkv_cache *cache, int32_t *offsets,
+                       int32_t *flat, cudaStream_t stream);
+
 /* Decode attention over the three tiers (implied by sec. 1 / sec. 5: attention runs
  * on the regularized layout). For each query head g of KV head h:
  *   out = sum_t softmax_t(l_t) v_t over

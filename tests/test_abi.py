@@ -113,6 +113,8 @@ def test_entry_points_validate_before_any_launch(lib):
                                            ctypes.c_float(0.9), 5, 0x300, ws, None) == B.EINVAL
     assert lib.hardkv_regularize(ctypes.byref(d), ctypes.byref(c), None, 0, ws, None) == B.EINVAL
     assert lib.hardkv_decode_attn(ctypes.byref(d), ctypes.byref(c), 0x100, None, ws, None) == B.EINVAL
+    assert lib.hardkv_flatten_sum(ctypes.byref(d), ctypes.byref(c), None, 0x200, None) == B.EINVAL
+    assert lib.hardkv_flatten_sum(ctypes.byref(d), ctypes.byref(c), 0x100, 0x204, None) == B.EALIGN
     bad = desc(dtype=9)
     assert lib.hardkv_condense(ctypes.byref(bad), ctypes.byref(c), ws, None) == B.EDTYPE
     assert lib.hardkv_decode_step(ctypes.byref(d), ctypes.byref(c), None, ws, None) == B.EINVAL

@@ -15,6 +15,7 @@ import torch
 from attention_kv_head_b200 import binding as B
 from attention_kv_head_b200 import synth
 from attention_kv_head_b200.cache import DecodeCache
+from oracle import hardkv_oracle as O
 from tests import gpu_util as U
 
 pytestmark = pytest.mark.gpu
@@ -191,3 +192,50 @@ def test_paged_pool_shortage_keeps_prefix():
     assert short_units > 0
     assert dc.read_status()[B.ST_FLAGS] & B.DEV_POOL_SHORT
     U.record("paged_shortage", short_units=short_units, **cmp.summary())
+
+
+@pytest.mark.parametrize("paged", [False, True], ids=["contiguous", "paged"])
+@pytest.mark.parametrize("name", ["bf16_ragged", "clamp", "f32_d64"])
+def test_flatten_sum_matches_oracle(name, paged):
+    """The sum form of the flattened index (offsets + flat list) against the oracle's
+    flatten_sum of the oracle units' own indices: before any selection (every count 0),
+    then after each of 6 steps under the MTI policy with reselection on block moves
+    (heads rewritten and heads loaded in place alike)."""
+    kw = {"bf16_ragged": dict(batch=5, context=None, len_range=(200, 700)),
+          "clamp": dict(sparse_cap=100),
+          "f32_d64": dict(dtype=synth.F32, n_q_heads=2, n_kv_heads=2, head_dim=64)}[name]
+    w = synth.small(steps=6, temp_range=(0.3, 6.0), **kw)
+    st = synth.initial_state(w)
+    pool = w.batch * w.n_kv_heads * tab_blocks(w) if paged else None
+    dc = DecodeCache.from_state(st, pool_blocks=pool)
+    units = [U.oracle_unit_from_state(st, b, h, steps=w.steps) for b in range(w.batch)
+             for h in range(w.n_kv_heads)]
+    cmp = U.StepCompare(w.dtype)
+    G, H = w.group, w.n_kv_heads
+    pol = layout(B.LAYOUT_MTI, l_lower=64, l_upper=300)
+    for t in range(-1, w.steps):
+        if t >= 0:
+            (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, t)
+            mask = dc.new_mask()
+            out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32,
+                              device=dc.device)
+            sm = B.SELECT_ALL if t == 0 else B.SELECT_MOVED
+            dc.step(q, k, v, out, w.p, mask=mask, layout=pol, select_mode=sm)
+            torch.cuda.synchronize()
+            m = mask.cpu().numpy().view(np.uint32)
+            for u, un in enumerate(units):
+                b, h = divmod(u, H)
+                res = un.step(q_ex[b, h * G:(h + 1) * G], k_ex[b, h], v_ex[b, h], 1.0, w.p,
+                              reselect="all" if t == 0 else "moved")
+                if res.sel is not None:
+                    kept = U.mask_bits(m[b, h], un.d_lo - un.s_lo)
+                    if not cmp.selection(res.sel, w.p, kept):
+                        U.adopt_selection(un, kept)
+        offsets, flat = dc.flatten_sum()
+        torch.cuda.synchronize()
+        want_off, want_flat = O.flatten_sum([un.idx[:un.n] for un in units])
+        got_off = offsets.cpu().numpy()
+        assert np.array_equal(got_off, want_off), t
+        assert np.array_equal(flat[:int(want_off[-1])].cpu().numpy(), want_flat), t
+    assert dc.read_status()[B.ST_FLAGS] == 0
+    U.record("flatten_sum", workload=name, paged=paged, **cmp.summary())
