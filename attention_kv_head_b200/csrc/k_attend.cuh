@@ -255,6 +255,7 @@ constexpr uint32_t kRowGather = 1u << 29, kRowIdx = (1u << 29) - 1;
 struct UnitView {
   Bounds bd;
   int n_u, nd, wgt;
+  int slo_row;   // ring row of position s_lo
   bool gather;   // reselected in this fused launch: kept rows come from the ring
   bool rewrite;  // Rewrite Cache layout (else Sparse Loading through sp_idx)
   const int32_t *spi;
@@ -282,7 +283,17 @@ __device__ __forceinline__ UnitView unit_view(const Shape &sh, const Cache &c, c
   v.spi = c.sp_idx + (size_t)u * sh.cap;
   v.wcd = c.w_cd + (size_t)u * sh.C;
   v.tab = c.k_pool ? c.blk_tab + (size_t)u * c.tab_blocks : nullptr;
+  v.slo_row = v.bd.ok ? v.bd.s_lo % sh.R : 0;
   return v;
+}
+
+// Ring row of a live position (s_lo <= pos < s_lo + R, which holds for every position a
+// valid unit reads: len - s_lo <= R): one wrap instead of a division.
+__device__ __forceinline__ uint32_t ring_row(const Shape &sh, const UnitView &v, int pos) {
+  int r = v.slo_row + (pos - v.bd.s_lo);
+  if (r >= sh.R) r -= sh.R;
+  if ((unsigned)r >= (unsigned)sh.R) r = ((pos % sh.R) + sh.R) % sh.R;  // not a live position
+  return (uint32_t)r;
 }
 
 // Row sources in two steps so the memory read can be issued ahead: row_fetch reads the
@@ -302,17 +313,17 @@ __device__ __forceinline__ uint32_t row_decode(const Shape &sh, const UnitView &
     if (v.gather) {
       if (pos >= v.bd.s_lo && pos < v.bd.d_lo) {
         bias = 0.f;
-        return kRowRing | (v.rewrite ? kRowGather : 0u) | (uint32_t)(pos % sh.R);
+        return kRowRing | (v.rewrite ? kRowGather : 0u) | ring_row(sh, v, pos);
       }
     } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | (uint32_t)(pos % sh.R));
+      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | ring_row(sh, v, pos));
     }
     return 0u;
   }
   if (j < v.n_u + v.nd) {
     bias = 0.f;
-    return kRowRing | (uint32_t)((v.bd.d_lo + (j - v.n_u)) % sh.R);
+    return kRowRing | ring_row(sh, v, v.bd.d_lo + (j - v.n_u));
   }
   const float wv = __uint_as_float(raw);
   if (wv > 0.f) {
@@ -330,17 +341,17 @@ __device__ __forceinline__ uint32_t row_code(const Shape &sh, const UnitView &v,
     if (v.gather) {
       if (pos >= v.bd.s_lo && pos < v.bd.d_lo) {
         bias = 0.f;
-        return kRowRing | (v.rewrite ? kRowGather : 0u) | (uint32_t)(pos % sh.R);
+        return kRowRing | (v.rewrite ? kRowGather : 0u) | ring_row(sh, v, pos);
       }
     } else if (pos >= v.bd.s_lo) {  // compact rows whose position was condensed are stale
       bias = 0.f;
-      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | (uint32_t)(pos % sh.R));
+      return v.rewrite ? (kRowCompact | compact_slot_row(v, j)) : (kRowRing | ring_row(sh, v, pos));
     }
     return 0u;
   }
   if (j < v.n_u + v.nd) {
     bias = 0.f;
-    return kRowRing | (uint32_t)((v.bd.d_lo + (j - v.n_u)) % sh.R);
+    return kRowRing | ring_row(sh, v, v.bd.d_lo + (j - v.n_u));
   }
   const int s = j - v.n_u - v.nd;
   const float wv = v.wcd[s];

@@ -98,7 +98,8 @@ __device__ __forceinline__ void ws_slice(WsState<D, NT> &st, const Shape &sh, co
       const float bias = i < 2 ? b0 : b8;
       x[i] = bias == -INFINITY ? -INFINITY : fmaf(sa[nt][i] + sb[nt][i], sl2, bias);
     }
-    float p[4];
+    float p[4], alpha[2];
+    bool grew = false;
 #pragma unroll
     for (int e = 0; e < 2; ++e) {  // query 2t + e: key rows g (x[e]) and g+8 (x[2+e])
       float mx = fmaxf(x[e], x[2 + e]);
@@ -106,19 +107,26 @@ __device__ __forceinline__ void ws_slice(WsState<D, NT> &st, const Shape &sh, co
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
       const float mn = fmaxf(st.m[nt][e], mx);
-      const float alpha = mn == -INFINITY ? 1.f : exp2f(st.m[nt][e] - mn);
+      grew |= mn > st.m[nt][e];
+      alpha[e] = mn == -INFINITY ? 1.f : exp2f(st.m[nt][e] - mn);
       p[e] = mn == -INFINITY ? 0.f : exp2f(x[e] - mn);
       p[2 + e] = mn == -INFINITY ? 0.f : exp2f(x[2 + e] - mn);
       float rs = p[e] + p[2 + e];
       rs += __shfl_xor_sync(0xffffffffu, rs, 4);
       rs += __shfl_xor_sync(0xffffffffu, rs, 8);
       rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-      st.l[nt][e] = st.l[nt][e] * alpha + rs;
+      st.l[nt][e] = st.l[nt][e] * alpha[e] + rs;
       st.m[nt][e] = mn;
+    }
+    // the accumulator is rescaled only when some query's running max rose (alpha = 1
+    // exactly otherwise, so skipping the multiply changes nothing)
+    if (__any_sync(0xffffffffu, grew)) {
 #pragma unroll
       for (int mt = 0; mt < D / 16; ++mt) {
-        st.o[nt][mt][e] *= alpha;
-        st.o[nt][mt][2 + e] *= alpha;
+        st.o[nt][mt][0] *= alpha[0];
+        st.o[nt][mt][1] *= alpha[1];
+        st.o[nt][mt][2] *= alpha[0];
+        st.o[nt][mt][3] *= alpha[1];
       }
     }
     // P^T (keys x queries) as the B operand: transpose the (key, query-pair) fragments
@@ -246,21 +254,26 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
       if (kind == kRowCond) return (kv ? vcd : kcd) + off;
       return nullptr;
     };
-    // copies of slice t into stage t % S: lane -> chunk cc of rows roff + k * RPI
+    // copies of slice t into stage t % S: lane -> chunk cc of rows roff + k * RPI. Each
+    // lane resolves the K / V addresses of its own row once (lane & 15); the chunk lanes
+    // of a row take them by shuffle.
     auto issue = [&](int t, const WsRow &rw) {
       if (t < ntiles) {
         uint8_t *dst = mine + (t % kWsStages) * Cfg::STAGE;
+        const unsigned long long mk = reinterpret_cast<unsigned long long>(src_of(rw.code, 0));
+        const unsigned long long mv = reinterpret_cast<unsigned long long>(src_of(rw.code, 1));
 #pragma unroll
         for (int k = 0; k < kWsRows / Cfg::RPI; ++k) {
           const int r = k * Cfg::RPI + roff;
-          const uint32_t code = __shfl_sync(0xffffffffu, rw.code, r);
-          const uint8_t *sk = src_of(code, 0), *sv = src_of(code, 1);
+          const uint8_t *sk = reinterpret_cast<const uint8_t *>(__shfl_sync(0xffffffffu, mk, r));
+          const uint8_t *sv = reinterpret_cast<const uint8_t *>(__shfl_sync(0xffffffffu, mv, r));
           cp_async16(dst + r * Cfg::STRIDE + cc * 16, sk ? sk + cc * 16 : kcd, sk ? 16 : 0);
           cp_async16(dst + Cfg::SLICE + r * Cfg::STRIDE + cc * 16, sv ? sv + cc * 16 : vcd, sv ? 16 : 0);
         }
       }
       cp_async_commit();  // one group per slice (possibly empty) keeps the count fixed
     };
+    const bool rewrite_now = v.gather && v.rewrite;  // this unit's kept rows are written
 
     WsState<D, NT> st;
     ws_state_init<D, NT>(st, sh, qp, u / sh.H, u % sh.H, lane);
@@ -273,27 +286,36 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
       issue(k, rows[k]);
     }
     for (int t = 0; t < ntiles; ++t) {
-      // slice t + S - 1 goes into the stage of slice t - 1 (computed last iteration)
+      // slice t + S - 1 goes into the stage of slice t - 1 (computed last iteration);
+      // that stage's bulk stores to the compact layout must have read it first
       const int tn = t + kWsStages - 1;
       rows[kWsStages - 1] = resolve(tn, raw_next);
       raw_next = fetch(tn + 1);
+      if (rewrite_now) {
+        bulk_wait_read<0>();
+        __syncwarp();
+      }
       issue(tn, rows[kWsStages - 1]);
       cp_async_wait<kWsStages - 1>();  // slice t has landed
-      __syncwarp();
       const uint8_t *ks = mine + (t % kWsStages) * Cfg::STAGE;
       const WsRow &cur = rows[0];
-      // Rewrite Cache: this slice's gathered rows -> compact slots (slot = union row)
-#pragma unroll
-      for (int k = 0; k < kWsRows / Cfg::RPI; ++k) {
-        const int r = k * Cfg::RPI + roff;
-        const uint32_t code = __shfl_sync(0xffffffffu, cur.code, r);
-        if (code & kRowGather) {
+      if (rewrite_now) {
+        // Rewrite Cache: this slice's gathered rows -> compact slots (slot = union row),
+        // one 1-D bulk copy per row: lane r < 16 the K row r, lane 16 + r the V row r
+        // (lanes 16..31 hold the codes of rows 0..15 too). The stage was written by
+        // every lane's cp.async (generic proxy): each lane fences its own writes for the
+        // async proxy before the warp meets.
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (cur.code & kRowGather) {
+          const int r = lane & 15;
           const size_t slot = compact_slot_row(v, r0 + t * kAttRows + w * kWsRows + r);
-          *reinterpret_cast<uint4 *>(ksp + slot * rb + cc * 16) =
-              *reinterpret_cast<const uint4 *>(ks + r * Cfg::STRIDE + cc * 16);
-          *reinterpret_cast<uint4 *>(vsp + slot * rb + cc * 16) =
-              *reinterpret_cast<const uint4 *>(ks + Cfg::SLICE + r * Cfg::STRIDE + cc * 16);
+          const int kv = lane >> 4;
+          bulk_s2g((kv ? vsp : ksp) + slot * rb, ks + kv * Cfg::SLICE + r * Cfg::STRIDE, (uint32_t)rb);
+          bulk_commit();
         }
+      } else {
+        __syncwarp();
       }
       const int g = lane >> 2;
       const float b0 = __shfl_sync(0xffffffffu, cur.bias, g);
@@ -304,6 +326,7 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
       for (int k = 0; k < kWsStages - 1; ++k) rows[k] = rows[k + 1];
     }
     cp_async_wait<0>();
+    bulk_wait<0>();   // this segment's compact rows are written and their sources read
     __syncthreads();  // every warp is done with its stages: reuse them as scratch
     ws_stage_state<D, NT>(st, sh, scratch, w, lane);
     merge_warps<D>(sh, ap, scratch, seg);
