@@ -428,8 +428,10 @@ __global__ void __launch_bounds__(kSelThreads)
   const int tm_stride = so.tm_stride;
   const float p = sp.p;
   const int u = blockIdx.x, b = u / sh.H;
-  pdl_wait();
-  pdl_launch();
+  // Before the dependency wait: what this kernel reads from the stages ahead of the
+  // score (boundaries and moves of the append, the caller's temperatures) is complete
+  // once this grid runs, because the score kernel releases it only after its own wait.
+  // Only the scores, tile maxima and entropy partials need the wait.
   if (!unit_active(select_mode, c.moved, b)) return;
   __shared__ SelShared S;
   __shared__ __align__(8) uint64_t fill_bar;
@@ -450,14 +452,10 @@ __global__ void __launch_bounds__(kSelThreads)
   const bool cached = L <= cache_n;
   const float *src = cached ? score_cache : sc;
 
-  // scores -> shared memory by one bulk copy (overlaps the max reduction); the row
-  // start is 256-byte aligned (R is a multiple of 64) and ceil4(L) <= R
   const uint32_t fill_bytes = (uint32_t)((L + 3) & ~3) * 4u;
   if (cached && L > 0 && tid == 0) {
     mbar_init(&fill_bar, 1);
     fence_barrier_init();
-    mbar_arrive_expect_tx(&fill_bar, fill_bytes);
-    bulk_g2s(score_cache, sc, fill_bytes, &fill_bar);
   }
   for (int i = tid; i < kBins; i += kSelThreads) {
     hcnt[i] = 0;
@@ -468,6 +466,14 @@ __global__ void __launch_bounds__(kSelThreads)
   if (tid == 0) {
     S.ncand = 0;
     S.n_keep = -1;
+  }
+  pdl_wait();
+  pdl_launch();
+  // scores -> shared memory by one bulk copy (overlaps the max reduction); the row
+  // start is 256-byte aligned (R is a multiple of 64) and ceil4(L) <= R
+  if (cached && L > 0 && tid == 0) {
+    mbar_arrive_expect_tx(&fill_bar, fill_bytes);
+    bulk_g2s(score_cache, sc, fill_bytes, &fill_bar);
   }
   // max score from the per-tile partial maxima (block_max synchronises)
   const TileSpan ts = tile_span(bd);
