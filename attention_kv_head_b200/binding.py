@@ -83,6 +83,8 @@ _SIGS = {
                                          _vp, _vp]),
     "hardkv_regularize_policy": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _i32,
                                                 ctypes.POINTER(LayoutPolicy), _vp, _vp]),
+    "hardkv_select_from_scores": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp,
+                                                 ctypes.c_float, _i32, _i32, _i32, _vp, _vp, _vp]),
     "hardkv_flatten_sum": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp, _vp]),
     "hardkv_decode_attn": (ctypes.c_int, [ctypes.POINTER(Desc), ctypes.POINTER(Cache), _vp, _vp,
                                           _vp, _vp]),

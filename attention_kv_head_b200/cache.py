@@ -157,6 +157,12 @@ class DecodeCache:
             self._c("hardkv_regularize_policy", _ptr(mask), select_mode, ctypes.byref(layout),
                     _ptr(self.ws), _stream(stream))
 
+    def select_from_scores(self, scores, p, mask, tau=None, rule=B.RULE_TOPP, top_k=0,
+                           select_mode=B.SELECT_ALL, stream=None):
+        """Calibrated top-p (or top-k) on caller importance scores [B,H,R] (float32)."""
+        self._c("hardkv_select_from_scores", _ptr(scores), _ptr(tau), ctypes.c_float(p), rule, top_k,
+                select_mode, _ptr(mask), _ptr(self.ws), _stream(stream))
+
     def flatten_sum(self, offsets=None, flat=None, stream=None):
         """Sum form of the flattened index: (offsets [B*H+1], flat [B*H*Cap]) int32;
         flat[offsets[u]:offsets[u+1]] is unit u's kept positions."""

@@ -443,11 +443,18 @@ int launch_score(const hardkv_desc *d, const Shape &sh, const Cache &c, const vo
   return HARDKV_OK;
 }
 
+// `given`: scores supplied by the caller ([B,H,R], no tile maxima) instead of the score
+// stage's output in the workspace.
 template <bool WRITE_IDX>
 int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, const SelectParams &sp,
                 int select_mode, uint32_t *mask, cudaStream_t st,
-                LayoutPolicy lp = LayoutPolicy{HARDKV_LAYOUT_REWRITE, 0, 0, 0, 0.f}) {
-  const ScoreOut so = score_out(ws, L, sp.ent != nullptr);
+                LayoutPolicy lp = LayoutPolicy{HARDKV_LAYOUT_REWRITE, 0, 0, 0, 0.f},
+                const float *given = nullptr) {
+  ScoreOut so = score_out(ws, L, sp.ent != nullptr);
+  if (given) {
+    so.scores = const_cast<float *>(given);
+    so.tile_max = nullptr;
+  }
   // the unit's scores are cached in shared memory when a whole ring fits
   const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
   const size_t smem = topp_smem_bytes(cache_n);
@@ -676,6 +683,27 @@ int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const 
   return launch_topp<false>(sh, c, ws, L,
                             select_params(nullptr, 1.0f, HARDKV_RULE_TOPK, k, false, nullptr, ws, L),
                             select_mode, mask, stream);
+}
+
+int hardkv_select_from_scores(const hardkv_desc *desc, const hardkv_cache *cache,
+                              const float *scores, const float *tau, float p, int32_t rule,
+                              int32_t top_k, int32_t select_mode, uint32_t *mask, void *ws,
+                              cudaStream_t stream) {
+  HKV_TRY(check_common(desc, cache, ws));
+  HKV_TRY(check_ptr(scores));
+  HKV_TRY(check_ptr(tau, true));
+  HKV_TRY(check_ptr(mask));
+  HKV_TRY(check_rule(desc, rule, top_k, HARDKV_CAL_TAU));
+  if (rule == HARDKV_RULE_TOPP) HKV_TRY(check_p(p));
+  HKV_TRY(check_mode(select_mode));
+  const Shape sh = make_shape(desc);
+  const Cache c = make_cache(desc, cache);
+  const Layout L = layout(desc);
+  return launch_topp<false>(sh, c, ws, L,
+                            select_params(tau, rule == HARDKV_RULE_TOPP ? p : 1.0f, rule, top_k, false,
+                                          nullptr, ws, L),
+                            select_mode, mask, stream, LayoutPolicy{HARDKV_LAYOUT_REWRITE, 0, 0, 0, 0.f},
+                            scores);
 }
 
 int hardkv_regularize(const hardkv_desc *desc, const hardkv_cache *cache, const uint32_t *mask,

@@ -478,11 +478,17 @@ __global__ void __launch_bounds__(kSelThreads)
   // max score from the per-tile partial maxima (block_max synchronises)
   const TileSpan ts = tile_span(bd);
   float m = -INFINITY;
-  for (int i = tid; i < ts.n * kPartsPerTile; i += kSelThreads)
-    m = fmaxf(m, tile_max[(size_t)u * tm_stride + i]);
-  const float M = block_max(m, S.red);  // also publishes fill_bar's initialisation
+  if (tile_max)
+    for (int i = tid; i < ts.n * kPartsPerTile; i += kSelThreads)
+      m = fmaxf(m, tile_max[(size_t)u * tm_stride + i]);
+  float M = block_max(m, S.red);  // also publishes fill_bar's initialisation
   if (cached && L > 0 && !mbar_wait(&fill_bar, 0) && tid == 0)
     flag(c.status, HARDKV_DEV_WAIT_TIMEOUT);
+  if (!tile_max) {  // scores from the caller come without maxima: reduce them here
+    m = -INFINITY;
+    for (int j = tid; j < L; j += kSelThreads) m = fmaxf(m, src[j]);
+    M = block_max(m, S.red);
+  }
   const bool topk = sp.rule == HARDKV_RULE_TOPK;
   if (sp.ent && !topk) tv = entropy_matched_tau(sh, sp, src, L, M, u, tm_stride, ts.n * kPartsPerTile, S);
   if (sp.tau_out && tid == 0) sp.tau_out[u] = topk ? 1.0f : tv;

@@ -272,6 +272,22 @@ int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const 
                       int32_t k, int32_t select_mode, uint32_t *mask, void *ws,
                       cudaStream_t stream);
 
+/* Stage 2b/2c on importance scores the caller supplies (any metric in place of the
+ * max-pooled logit: sec. 2.B calibrates "scores" into one probability space, whatever
+ * produced them). scores: device float [B,H,R], candidate j of (b,h) (position
+ * s_lo + j, j < d_lo - s_lo) at scores[(b*H + h)*R + j], 16-byte aligned; other entries
+ * are not read. rule HARDKV_RULE_TOPP: calibrated top-p with tau (device float [B,H] or
+ * NULL = 1) and 0 < p <= 1, at most Cap kept, exactly as hardkv_score_calibrate_topp
+ * after its score stage; HARDKV_RULE_TOPK: the top_k best (1 <= top_k <= Cap; p and
+ * tau unused). The head's maximum is taken from the scores themselves. mask as in
+ * hardkv_score_calibrate_topp; pass it to hardkv_regularize(_policy) to finish stage 3.
+ * Scores must be finite: non-finite ones are not checked and select unspecified
+ * candidates (every access stays in bounds). */
+int hardkv_select_from_scores(const hardkv_desc *desc, const hardkv_cache *cache,
+                              const float *scores, const float *tau, float p, int32_t rule,
+                              int32_t top_k, int32_t select_mode, uint32_t *mask, void *ws,
+                              cudaStream_t stream);
+
 /* Stage 3 (sec. 2.C Index Regularization: Rewrite Cache + Flatten Index to the max
  * length). For each selected (b,h): the kept candidates of `mask` (device, layout as
  * above), in ascending position order, go to compact slots 0..n-1 — K and V rows

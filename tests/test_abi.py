@@ -113,6 +113,21 @@ def test_entry_points_validate_before_any_launch(lib):
                                            ctypes.c_float(0.9), 5, 0x300, ws, None) == B.EINVAL
     assert lib.hardkv_regularize(ctypes.byref(d), ctypes.byref(c), None, 0, ws, None) == B.EINVAL
     assert lib.hardkv_decode_attn(ctypes.byref(d), ctypes.byref(c), 0x100, None, ws, None) == B.EINVAL
+    sel = lib.hardkv_select_from_scores
+    assert sel(ctypes.byref(d), ctypes.byref(c), None, None, ctypes.c_float(0.9), B.RULE_TOPP, 0, 0,
+               0x300, ws, None) == B.EINVAL                      # no scores
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x104, None, ctypes.c_float(0.9), B.RULE_TOPP, 0, 0,
+               0x300, ws, None) == B.EALIGN                      # misaligned scores
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x100, 0x204, ctypes.c_float(0.9), B.RULE_TOPP, 0, 0,
+               0x300, ws, None) == B.EALIGN                      # misaligned tau
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x100, None, ctypes.c_float(0.0), B.RULE_TOPP, 0, 0,
+               0x300, ws, None) == B.EINVAL                      # p out of range
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x100, None, ctypes.c_float(0.9), B.RULE_TOPK, 0, 0,
+               0x300, ws, None) == B.EINVAL                      # k out of range
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x100, None, ctypes.c_float(0.9), 7, 1, 0,
+               0x300, ws, None) == B.EINVAL                      # unknown rule
+    assert sel(ctypes.byref(d), ctypes.byref(c), 0x100, None, ctypes.c_float(0.9), B.RULE_TOPP, 0, 3,
+               0x300, ws, None) == B.EINVAL                      # unknown select mode
     assert lib.hardkv_flatten_sum(ctypes.byref(d), ctypes.byref(c), None, 0x200, None) == B.EINVAL
     assert lib.hardkv_flatten_sum(ctypes.byref(d), ctypes.byref(c), 0x100, 0x204, None) == B.EALIGN
     bad = desc(dtype=9)
