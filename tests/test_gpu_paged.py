@@ -239,3 +239,64 @@ def test_flatten_sum_matches_oracle(name, paged):
         assert np.array_equal(flat[:int(want_off[-1])].cpu().numpy(), want_flat), t
     assert dc.read_status()[B.ST_FLAGS] == 0
     U.record("flatten_sum", workload=name, paged=paged, **cmp.summary())
+
+
+def test_full_size_paged_step_and_sum_form():
+    """llama8b_8k at full size (64 heads, 7680 candidates each): one fused step on a
+    paged and on a contiguous cache gives bit-identical outputs, masks, indices and
+    compact rows, the pool is a partition, and the sum form of the flattened index holds
+    at any size: offsets are the running kept counts and each head's slice of the flat
+    list is its max-length row up to n_kept."""
+    w = synth.WORKLOADS["llama8b_8k"]
+    st = synth.initial_state(w)
+    dc0 = DecodeCache.from_state(st)
+    dc1 = DecodeCache.from_state(st, pool_blocks=w.batch * w.n_kv_heads * tab_blocks(w))
+    (q, k, v), _ = U.upload_step(dc0, w, st, 0)
+    outs, masks = [], []
+    for dc in (dc0, dc1):
+        mask = dc.new_mask()
+        out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
+        dc.step(q, k, v, out, w.p, mask=mask)
+        outs.append(out)
+        masks.append(mask)
+    torch.cuda.synchronize()
+    assert torch.equal(masks[0], masks[1]) and torch.equal(outs[0], outs[1])
+    assert_same_compact(dc0, dc1)
+    for dc in (dc0, dc1):
+        offsets, flat = dc.flatten_sum()
+        torch.cuda.synchronize()
+        n = dc.n_kept.cpu().numpy().reshape(-1).astype(np.int64)
+        off = offsets.cpu().numpy()
+        assert np.array_equal(off, np.concatenate([[0], np.cumsum(n)]))
+        idx = dc.sp_idx.cpu().numpy().reshape(n.size, -1)
+        fl = flat.cpu().numpy()
+        for u in range(n.size):
+            assert np.array_equal(fl[off[u]:off[u + 1]], idx[u, :n[u]]), u
+        assert dc.read_status()[B.ST_FLAGS] == 0
+
+
+@pytest.mark.parametrize("sel", ["topk", "entropy"])
+def test_paged_steps_other_rules(sel):
+    """The block manager is independent of how the selection was made: 12 fused steps
+    with the fixed top-k rule, and with the entropy-matched temperature, bit-identical on
+    the paged and the contiguous cache."""
+    w = synth.small(condense_mode=synth.MERGE, steps=12, batch=2, context=300, p=0.8,
+                    temp_range=(0.3, 6.0))
+    st = synth.initial_state(w)
+    dc0 = DecodeCache.from_state(st)
+    dc1 = DecodeCache.from_state(st, pool_blocks=w.batch * w.n_kv_heads * tab_blocks(w))
+    kw = dict(rule=B.RULE_TOPK, top_k=90) if sel == "topk" else dict(calibration=B.CAL_ENTROPY)
+    for t in range(w.steps):
+        (q, k, v), _ = U.upload_step(dc0, w, st, t)
+        outs, masks = [], []
+        for dc in (dc0, dc1):
+            mask = dc.new_mask()
+            out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32,
+                              device=dc.device)
+            dc.step(q, k, v, out, w.p, mask=mask, **kw)
+            outs.append(out)
+            masks.append(mask)
+        torch.cuda.synchronize()
+        assert torch.equal(masks[0], masks[1]) and torch.equal(outs[0], outs[1]), t
+        assert_same_compact(dc0, dc1)
+    assert dc1.read_status()[B.ST_FLAGS] == 0
