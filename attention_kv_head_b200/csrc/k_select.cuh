@@ -529,8 +529,9 @@ __global__ void __launch_bounds__(kSelThreads)
       hmass[i] = (unsigned long long)hpart[i] +
                  ((unsigned long long)hpart[kBins + i] << kPartBits) +
                  ((unsigned long long)hpart[2 * kBins + i] << (2 * kPartBits));
-    unsigned long long Z = 0;
-    for (int w = 0; w < kSelThreads / 32; ++w) Z += S.wmass[w];
+    unsigned long long Z = S.wmass[lane];  // every warp sums the 32 warp totals
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
     __syncthreads();
     // the threshold T = ceil(p Z) (p >= 1 keeps all, up to Cap; top-k has no mass rule)
     if (p < 1.0f && !topk) T = (unsigned long long)ceil((double)p * (double)Z);
@@ -569,8 +570,9 @@ __global__ void __launch_bounds__(kSelThreads)
     __syncthreads();
     const int ncand = S.ncand;
     if (!use_cnt) {
-      above_cnt = 0;
-      for (int w = 0; w < kSelThreads / 32; ++w) above_cnt += (uint32_t)S.scan[w];
+      above_cnt = (uint32_t)S.scan[lane];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) above_cnt += __shfl_xor_sync(0xffffffffu, above_cnt, o);
     }
     if (ncand <= 64) {
       // small bins: one warp sorts the candidates and finds the cut (no block barrier)
