@@ -1,6 +1,8 @@
 // Stage 2b/2c: Logits Calibration + calibrated top-p (HARD-KV technical summary sec.
-// 2.B, sec. 2.A Tier 2) and stage 3, Index Regularization by prefix scan (sec. 2.C
-// Rewrite Cache, Flatten Index to the maximum length).
+// 2.B, sec. 2.A Tier 2), also on caller-supplied scores and with the fixed top-k rule,
+// and stage 3, Index Regularization by prefix scan (sec. 2.C Rewrite Cache, Sparse
+// Loading, Flatten Index to the maximum length and, on demand, to the sum); the paged
+// tier's block allocation happens inside the selecting launch (common.cuh pool_assign).
 //
 // Top-p without a sort: the calibrated mass of candidate j is
 //   m_j = exp((s_j - max s) / tau)      (unnormalised; the threshold is p * sum m)

@@ -11,8 +11,11 @@
  * and runs every decode step through four stages (sec. 2.A): (1) linear append
  * to Dense; (2) Logits Calibration + top-p -> selection masks; (3) Index
  * Regularization: kept rows rewritten into a contiguous fixed-capacity layout
- * (sec. 2.C Rewrite Cache, Flatten Index to the maximum length); (4) eviction or
- * weighted merge of the oldest block; then decode attention over the tiers.
+ * (sec. 2.C Rewrite Cache, Flatten Index to the maximum length) or only indexed
+ * (Sparse Loading), per head by a layout policy; the index also in its sum form on
+ * demand, the rewritten rows optionally in a shared pool of 16-row blocks (sec. 2.C
+ * head-wise block manager); (4) eviction or weighted merge of the oldest block; then
+ * decode attention over the tiers.
  *
  * Conventions for every entry point:
  *  - Pointers marked "device" are CUDA device pointers owned by the caller; the
@@ -26,7 +29,7 @@
  *    bfloat16). Attention output is float32.
  *  - Layouts are row-major, innermost dimension last:
  *      ring K/V  [B, H, R, d]   position p of unit (b,h) lives in row p mod R
- *      compact   [B, H, Cap, d] slots 0..n-1 valid
+ *      compact   [B, H, Cap, d] slots 0..n-1 valid (or pool blocks: hardkv_cache)
  *      condensed [B, H, C, d]   weights [B, H, C] float32 (0 = empty slot)
  *      q [B, Hq, d]; query head qh belongs to KV head qh / (Hq / H)
  *  - Return value: HARDKV_OK (0) or a negative HARDKV_E* code. Arguments are
