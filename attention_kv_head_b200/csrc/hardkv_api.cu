@@ -360,15 +360,20 @@ int resident_ctas_cached(K kernel, int threads, size_t smem) {
   return n;
 }
 
+// q_src / q_dst: queries the append kernel also copies (NULL: none)
 int launch_append(const hardkv_desc *d, const Shape &sh, const Cache &c, const void *k_new,
-                  const void *v_new, void *ws, const Layout &L, cudaStream_t st) {
+                  const void *v_new, void *ws, const Layout &L, cudaStream_t st,
+                  const void *q_src = nullptr, void *q_dst = nullptr) {
   int *counters = reinterpret_cast<int *>(static_cast<char *>(ws) + L.counters);
   if (d->dtype == HARDKV_BF16)
     append_kernel<bf16><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const bf16 *>(k_new),
-                                              static_cast<const bf16 *>(v_new), counters);
+                                              static_cast<const bf16 *>(v_new), counters,
+                                              static_cast<const bf16 *>(q_src), static_cast<bf16 *>(q_dst));
   else
     append_kernel<float><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const float *>(k_new),
-                                               static_cast<const float *>(v_new), counters);
+                                               static_cast<const float *>(v_new), counters,
+                                               static_cast<const float *>(q_src),
+                                               static_cast<float *>(q_dst));
   HKV_CHECK_LAUNCH("append_kernel");
   return HARDKV_OK;
 }
@@ -747,8 +752,11 @@ int hardkv_decode_attn(const hardkv_desc *desc, const hardkv_cache *cache, const
                        stream);
 }
 
-int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
-                       const hardkv_step_args *a, void *ws, cudaStream_t stream) {
+// The fused step. q_host: the caller's queries in mapped host memory, copied to a->q by
+// the append kernel (host entry point), or NULL (a->q already on the device).
+static int decode_step_impl(const hardkv_desc *desc, const hardkv_cache *cache,
+                            const hardkv_step_args *a, void *ws, cudaStream_t stream,
+                            const void *q_host) {
   HKV_TRY(check_common(desc, cache, ws));
   HKV_TRY(check_step_args(a, false));
   HKV_TRY(check_rule(desc, a->rule, a->top_k, a->calibration));
@@ -763,7 +771,8 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   if (tma) HKV_TRY(make_kmap(&kmap, desc, c.k_ring));  // host work before the first launch
   cudaEvent_t *ev = a->stage_events;
   HKV_TRY(record(ev, 0, stream));
-  HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, ws, L, stream));  // zeroes counters
+  HKV_TRY(launch_append(desc, sh, c, a->k_new, a->v_new, ws, L, stream, q_host,
+                        q_host ? const_cast<void *>(a->q) : nullptr));  // zeroes counters
   HKV_TRY(record(ev, 1, stream));
   HKV_TRY(launch_condense(desc, sh, c, stream));
   HKV_TRY(record(ev, 2, stream));
@@ -776,6 +785,11 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
   HKV_TRY(record(ev, 4, stream));
   HKV_TRY(launch_attend(desc, sh, c, a->q, a->out, ws, L, 1, a->select_mode, false, stream));
   return record(ev, 5, stream);
+}
+
+int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
+                       const hardkv_step_args *a, void *ws, cudaStream_t stream) {
+  return decode_step_impl(desc, cache, a, ws, stream, nullptr);
 }
 
 // Device address of a host buffer the GPU can reach in place (pinned and mapped, as
@@ -811,16 +825,19 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   dv.v_new = w + L.st_v;
   dv.out = reinterpret_cast<float *>(w + L.st_out);
   dv.tau = h->tau ? reinterpret_cast<const float *>(w + L.st_tau) : nullptr;
-  // q is read by many CTAs and is copied; k_new / v_new (read once, by the append
-  // kernel) and out (written once per unit) are used in place when the GPU can address
-  // them, which saves three copy latencies per step; other host memory is staged
+  // k_new / v_new (read once, by the append kernel) and out (written once per unit) are
+  // used in place when the GPU can address them; q, read by many CTAs, goes to the
+  // device staging buffer: copied by the append kernel itself when the GPU can address
+  // it, else by a copy. That saves four copy latencies per step; other host memory is
+  // staged by copies.
   void *k_map = mapped_host(h->k_new), *v_map = mapped_host(h->v_new);
-  void *o_map = mapped_host(h->out);
+  void *o_map = mapped_host(h->out), *q_map = mapped_host(h->q);
   if (k_map) dv.k_new = k_map;
   if (v_map) dv.v_new = v_map;
   if (o_map) dv.out = static_cast<float *>(o_map);
   cudaError_t r;
-  if ((r = cudaMemcpyAsync(w + L.st_q, h->q, nq * e, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+  if ((!q_map &&
+       (r = cudaMemcpyAsync(w + L.st_q, h->q, nq * e, cudaMemcpyHostToDevice, stream)) != cudaSuccess) ||
       (!k_map && (r = cudaMemcpyAsync(w + L.st_k, h->k_new, U * desc->head_dim * e,
                                       cudaMemcpyHostToDevice, stream)) != cudaSuccess) ||
       (!v_map && (r = cudaMemcpyAsync(w + L.st_v, h->v_new, U * desc->head_dim * e,
@@ -829,7 +846,7 @@ int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
   if (h->tau && (r = cudaMemcpyAsync(w + L.st_tau, h->tau, U * 4, cudaMemcpyHostToDevice, stream)) !=
                     cudaSuccess)
     return cuda_fail(r, "cudaMemcpyAsync H2D");
-  HKV_TRY(hardkv_decode_step(desc, cache, &dv, ws, stream));
+  HKV_TRY(decode_step_impl(desc, cache, &dv, ws, stream, q_map));
   if (!o_map && (r = cudaMemcpyAsync(h->out, w + L.st_out, nq * 4, cudaMemcpyDeviceToHost, stream)) !=
                     cudaSuccess)
     return cuda_fail(r, "cudaMemcpyAsync D2H");

@@ -8,13 +8,22 @@ namespace hardkv {
 
 // One CTA per sequence b (so the per-sequence boundary update has one writer).
 // Copies k_new/v_new [B,H,d] into ring row len mod R, then advances the boundaries.
+// q_src != NULL: also copies this sequence's queries q_src[b] -> q_dst[b] ([B,Hq,d]; the
+// host entry point's queries, read in place from mapped host memory).
 template <typename T>
 __global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T *k_new,
-                                                     const T *v_new, int *counters) {
+                                                     const T *v_new, int *counters,
+                                                     const T *q_src, T *q_dst) {
   const int b = blockIdx.x;
   pdl_wait();  // the previous step's kernels finish before this one touches the state
   pdl_launch();
   if (b == 0 && c.k_pool) pool_merge(c);  // blocks returned last step become free
+  if (q_src) {
+    const int nq = sh.Hq * sh.d * (int)sizeof(T) / 16;  // 16-byte vectors of q[b]
+    const uint4 *qs = reinterpret_cast<const uint4 *>(q_src + (size_t)b * sh.Hq * sh.d);
+    uint4 *qd = reinterpret_cast<uint4 *>(q_dst + (size_t)b * sh.Hq * sh.d);
+    for (int i = threadIdx.x; i < nq; i += blockDim.x) qd[i] = qs[i];
+  }
   // attention completion counters of this sequence's units start the step at zero
   if (counters)
     for (int h = threadIdx.x; h < sh.H; h += blockDim.x) counters[b * sh.H + h] = 0;

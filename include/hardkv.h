@@ -351,8 +351,9 @@ int hardkv_decode_step(const hardkv_desc *desc, const hardkv_cache *cache,
  * args->tau_out, if not NULL, are device pointers. Every argument is checked before
  * the first copy is enqueued. Staging buffers live in the workspace. Pinned, mapped
  * and 16-byte aligned k_new, v_new and out buffers (cudaHostAlloc memory under
- * unified addressing) are read / written by the kernels in place instead of copied;
- * q and tau are always copied. */
+ * unified addressing) are read / written by the kernels in place instead of copied,
+ * and such a q is copied to its staging buffer by the first kernel of the step (one
+ * copy fewer on the stream); tau is always copied. */
 int hardkv_decode_step_host(const hardkv_desc *desc, const hardkv_cache *cache,
                             const hardkv_step_args *host_args, void *ws,
                             cudaStream_t stream);
