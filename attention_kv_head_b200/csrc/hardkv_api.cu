@@ -366,11 +366,11 @@ int launch_append(const hardkv_desc *d, const Shape &sh, const Cache &c, const v
                   const void *q_src = nullptr, void *q_dst = nullptr) {
   int *counters = reinterpret_cast<int *>(static_cast<char *>(ws) + L.counters);
   if (d->dtype == HARDKV_BF16)
-    append_kernel<bf16><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const bf16 *>(k_new),
+    append_kernel<bf16><<<sh.B, kAppendThreads, 0, st>>>(sh, c, static_cast<const bf16 *>(k_new),
                                               static_cast<const bf16 *>(v_new), counters,
                                               static_cast<const bf16 *>(q_src), static_cast<bf16 *>(q_dst));
   else
-    append_kernel<float><<<sh.B, 128, 0, st>>>(sh, c, static_cast<const float *>(k_new),
+    append_kernel<float><<<sh.B, kAppendThreads, 0, st>>>(sh, c, static_cast<const float *>(k_new),
                                                static_cast<const float *>(v_new), counters,
                                                static_cast<const float *>(q_src),
                                                static_cast<float *>(q_dst));

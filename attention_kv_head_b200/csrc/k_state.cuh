@@ -6,12 +6,15 @@
 
 namespace hardkv {
 
-// One CTA per sequence b (so the per-sequence boundary update has one writer).
+// One CTA per sequence b (so the per-sequence boundary update has one writer); 512
+// threads so that all of a sequence's rows are in flight at once (the host entry point's
+// k_new, v_new and q come over the host link, where each round trip costs microseconds).
+constexpr int kAppendThreads = 512;
 // Copies k_new/v_new [B,H,d] into ring row len mod R, then advances the boundaries.
 // q_src != NULL: also copies this sequence's queries q_src[b] -> q_dst[b] ([B,Hq,d]; the
 // host entry point's queries, read in place from mapped host memory).
 template <typename T>
-__global__ void __launch_bounds__(128) append_kernel(Shape sh, Cache c, const T *k_new,
+__global__ void __launch_bounds__(kAppendThreads) append_kernel(Shape sh, Cache c, const T *k_new,
                                                      const T *v_new, int *counters,
                                                      const T *q_src, T *q_dst) {
   const int b = blockIdx.x;
