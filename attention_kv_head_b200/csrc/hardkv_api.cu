@@ -157,7 +157,7 @@ int check_cache(const hardkv_cache *c) {
     if (!aligned16(p)) return HARDKV_EALIGN;
   }
   // pool rows are addressed by 29-bit row codes and 32-bit block ids
-  if (c->pool_blocks < 1 || c->pool_blocks * HARDKV_PAGE_ROWS >= (int64_t(1) << 29))
+  if (c->pool_blocks < 1 || c->pool_blocks >= ((int64_t(1) << 29) / HARDKV_PAGE_ROWS))
     return HARDKV_EINVAL;
   return HARDKV_OK;
 }

@@ -156,7 +156,7 @@ def test_paged_cache_validates(lib):
     for name in POOL_FIELDS:
         assert append(_fake_cache(paged=True, null=name)) == B.EINVAL, name
         assert append(_fake_cache(paged=True, misalign=name)) == B.EALIGN, name
-    for blocks in (0, -1, (1 << 29) // B.PAGE_ROWS):
+    for blocks in (0, -1, (1 << 29) // B.PAGE_ROWS, 1 << 62):
         c = _fake_cache(paged=True)
         c.pool_blocks = blocks
         assert append(c) == B.EINVAL, blocks
