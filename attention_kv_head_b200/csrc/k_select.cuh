@@ -19,6 +19,7 @@
 namespace hardkv {
 
 constexpr int kSelThreads = 1024;
+constexpr int kLoadBatch = 8;  // scores a thread loads ahead in the element passes
 constexpr float kMassScale = 1099511627776.0f;  // 2^40
 
 // Exclusive scan of a 0/1 flag over a 1024-thread block; returns (excl, total).
@@ -420,8 +421,10 @@ __global__ void __launch_bounds__(128) pool_alloc_kernel(Shape sh, Cache c, cons
 // (key desc, position asc) and cut by a prefix sum of their masses; larger bins fall
 // back to a radix select (11 + 11 + 10 key bits). The result is the pair
 // (theta, pos_cut): candidate j is kept iff key_j > theta, or key_j == theta and
-// j <= pos_cut.
-template <bool WRITE_IDX>
+// j <= pos_cut. CACHED: the row's scores are copied to shared memory (cache_n = R
+// floats); otherwise every pass reads them from global memory (L2). One instance per
+// case keeps each kernel's code to the path it runs.
+template <bool WRITE_IDX, bool CACHED>
 __global__ void __launch_bounds__(kSelThreads)
     topp_kernel(Shape sh, Cache c, ScoreOut so, SelectParams sp, int select_mode,
                 uint32_t *__restrict__ mask, int cache_n, LayoutPolicy lp) {
@@ -451,7 +454,7 @@ __global__ void __launch_bounds__(kSelThreads)
   const int L = bd.ok ? bd.d_lo - bd.s_lo : 0;
   const float *sc = scores + (size_t)u * sh.R;
   float tv = sp.tau ? sp.tau[u] : 1.0f;
-  const bool cached = L <= cache_n;
+  constexpr bool cached = CACHED;  // L <= R = cache_n
   const float *src = cached ? score_cache : sc;
 
   const uint32_t fill_bytes = (uint32_t)((L + 3) & ~3) * 4u;
@@ -508,9 +511,7 @@ __global__ void __launch_bounds__(kSelThreads)
   if (!keep_all) {
     // level 1: per-bin count and mass; the thread's own mass total for Z
     unsigned long long zt = 0;
-#pragma unroll 4
-    for (int j = tid; j < L; j += kSelThreads) {
-      const float s = src[j];
+    auto level1_one = [&](float s) {
       const int bin = bin_of(s);
       const unsigned long long mf = mass_fx(s, M, tv);
       zt += mf;
@@ -522,6 +523,24 @@ __global__ void __launch_bounds__(kSelThreads)
       if (p0) atomicAdd(&hpart[bin], p0);
       if (p1) atomicAdd(&hpart[kBins + bin], p1);
       if (p2) atomicAdd(&hpart[2 * kBins + bin], p2);
+    };
+    if constexpr (CACHED) {
+#pragma unroll 4
+      for (int j = tid; j < L; j += kSelThreads) level1_one(src[j]);
+    } else {
+      // scores from L2 (a row too long for shared memory): kLoadBatch per thread are
+      // loaded before any is used, so that many loads are in flight
+      for (int j0 = tid; j0 < L; j0 += kLoadBatch * kSelThreads) {
+        float sv[kLoadBatch];
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i) {
+          const int j = j0 + i * kSelThreads;
+          sv[i] = j < L ? src[j] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i)
+          if (j0 + i * kSelThreads < L) level1_one(sv[i]);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) zt += __shfl_xor_sync(0xffffffffu, zt, o);
@@ -550,9 +569,9 @@ __global__ void __launch_bounds__(kSelThreads)
     // candidates: the elements of bin b1 (every element with the threshold key is one);
     // without per-bin counts, also the number of elements above b1
     uint32_t n_above = 0;
-    for (int j0 = 0; j0 < L; j0 += kSelThreads) {
+    // one block-wide row of candidates starting at j0 (uniform); s = this thread's score
+    auto cand_row = [&](int j0, float s) {
       const int j = j0 + tid;
-      const float s = j < L ? src[j] : 0.f;
       const int bn = j < L ? bin_of(s) : kBins;
       const bool member = bn == b1;
       if (!use_cnt) n_above += __popc(__ballot_sync(0xffffffffu, bn < b1));
@@ -566,6 +585,21 @@ __global__ void __launch_bounds__(kSelThreads)
           ckey[k] = order_key(s);
           cpos[k] = j;
         }
+      }
+    };
+    if constexpr (CACHED) {
+      for (int j0 = 0; j0 < L; j0 += kSelThreads) cand_row(j0, j0 + tid < L ? src[j0 + tid] : 0.f);
+    } else {
+      for (int jb = 0; jb < L; jb += kLoadBatch * kSelThreads) {
+        float sv[kLoadBatch];  // this thread's scores of the batch, loaded first
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i) {
+          const int j = jb + i * kSelThreads + tid;
+          sv[i] = j < L ? src[j] : 0.f;
+        }
+#pragma unroll
+        for (int i = 0; i < kLoadBatch; ++i)
+          if (jb + i * kSelThreads < L) cand_row(jb + i * kSelThreads, sv[i]);  // uniform
       }
     }
     if (!use_cnt && lane == 0) S.scan[warp] = (int)n_above;
@@ -813,26 +847,46 @@ __global__ void __launch_bounds__(kSelThreads)
       }
     }
   } else {
+    // long rows: the words are kept in the histogram's shared memory (free once the cut
+    // is known; nwords <= kMaxSelectRows / 32 = 8192 words fits its 48 KB), so the index
+    // pass reads them instead of the scores; the scores come kLoadBatch per lane at once
+    uint32_t *wbuf = reinterpret_cast<uint32_t *>(hmass);  // hmass, hcnt, hpart: 48 KB in a row
     int wcount = 0;
-    for (int k = 0; k < K; ++k) {
-      const int wi = warp * K + k;
-      if (wi >= nwords) break;
-      const unsigned word = __ballot_sync(0xffffffffu, kept_at(wi * 32 + lane));
-      if (mrow && lane == 0) mrow[wi] = word;
-      wcount += __popc(word);
+    for (int k0 = 0; k0 < K; k0 += kLoadBatch) {
+      float sv[kLoadBatch];
+#pragma unroll
+      for (int i = 0; i < kLoadBatch; ++i) {
+        const int j = (warp * K + k0 + i) * 32 + lane;
+        sv[i] = (k0 + i < K && j < L) ? src[j] : 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < kLoadBatch; ++i) {
+        const int wi = warp * K + k0 + i;
+        if (k0 + i >= K || wi >= nwords) break;  // uniform over the warp
+        const int j = wi * 32 + lane;
+        bool kept = false;
+        if (j < L) {
+          const uint32_t key = order_key(sv[i]);
+          kept = key > theta || (key == theta && j <= pos_cut);
+        }
+        const unsigned word = __ballot_sync(0xffffffffu, kept);
+        if (lane == 0) {
+          if (mrow) mrow[wi] = word;
+          wbuf[wi] = word;
+        }
+        wcount += __popc(word);
+      }
     }
     if (WRITE_IDX) {
       if (lane == 0) S.scan[warp] = wcount;
-      __syncthreads();
+      __syncthreads();  // also publishes wbuf
       int base = warp_prefix_of(S.scan, warp, lane);
       for (int k = 0; k < K; ++k) {
         const int wi = warp * K + k;
         if (wi >= nwords) break;
-        const int j = wi * 32 + lane;
-        const bool kept = kept_at(j);
-        const unsigned word = __ballot_sync(0xffffffffu, kept);
+        const unsigned word = wbuf[wi];
         const int slot = base + __popc(word & lt_mask);
-        if (kept && slot < n) idx[slot] = bd.s_lo + j;
+        if (((word >> lane) & 1u) && slot < n) idx[slot] = bd.s_lo + wi * 32 + lane;
         base += __popc(word);
       }
     }
