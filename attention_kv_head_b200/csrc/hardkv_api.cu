@@ -463,15 +463,19 @@ int launch_topp(const Shape &sh, const Cache &c, void *ws, const Layout &L, cons
   // the unit's scores are cached in shared memory when a whole ring fits
   const int cache_n = sh.R <= kToppCacheMax ? sh.R : 0;
   const size_t smem = topp_smem_bytes(cache_n);
-  if (cache_n > 0) {
-    HKV_TRY(set_smem(topp_kernel<WRITE_IDX, true>, smem));
-    launch_pdl(topp_kernel<WRITE_IDX, true>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, so,
-               sp, select_mode, mask, cache_n, lp);
-  } else {
-    HKV_TRY(set_smem(topp_kernel<WRITE_IDX, false>, smem));
-    launch_pdl(topp_kernel<WRITE_IDX, false>, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, so,
-               sp, select_mode, mask, cache_n, lp);
-  }
+  auto go = [&](auto kernel) -> int {
+    HKV_TRY(set_smem(kernel, smem));
+    launch_pdl(kernel, dim3(sh.B * sh.H), dim3(kSelThreads), smem, st, sh, c, so, sp, select_mode, mask,
+               cache_n, lp);
+    return HARDKV_OK;
+  };
+  const bool ent = sp.ent != nullptr;
+  int rc;
+  if (cache_n > 0)
+    rc = ent ? go(topp_kernel<WRITE_IDX, true, true>) : go(topp_kernel<WRITE_IDX, true, false>);
+  else
+    rc = ent ? go(topp_kernel<WRITE_IDX, false, true>) : go(topp_kernel<WRITE_IDX, false, false>);
+  HKV_TRY(rc);
   HKV_CHECK_LAUNCH("topp_kernel");
   return HARDKV_OK;
 }

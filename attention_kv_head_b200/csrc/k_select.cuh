@@ -423,8 +423,9 @@ __global__ void __launch_bounds__(128) pool_alloc_kernel(Shape sh, Cache c, cons
 // (theta, pos_cut): candidate j is kept iff key_j > theta, or key_j == theta and
 // j <= pos_cut. CACHED: the row's scores are copied to shared memory (cache_n = R
 // floats); otherwise every pass reads them from global memory (L2). One instance per
-// case keeps each kernel's code to the path it runs.
-template <bool WRITE_IDX, bool CACHED>
+// case keeps each kernel's code to the path it runs; likewise ENT (the entropy-matched
+// temperature solve, used when sp.ent is set).
+template <bool WRITE_IDX, bool CACHED, bool ENT>
 __global__ void __launch_bounds__(kSelThreads)
     topp_kernel(Shape sh, Cache c, ScoreOut so, SelectParams sp, int select_mode,
                 uint32_t *__restrict__ mask, int cache_n, LayoutPolicy lp) {
@@ -495,7 +496,8 @@ __global__ void __launch_bounds__(kSelThreads)
     M = block_max(m, S.red);
   }
   const bool topk = sp.rule == HARDKV_RULE_TOPK;
-  if (sp.ent && !topk) tv = entropy_matched_tau(sh, sp, src, L, M, u, tm_stride, ts.n * kPartsPerTile, S);
+  if constexpr (ENT)
+    if (sp.ent && !topk) tv = entropy_matched_tau(sh, sp, src, L, M, u, tm_stride, ts.n * kPartsPerTile, S);
   if (sp.tau_out && tid == 0) sp.tau_out[u] = topk ? 1.0f : tv;
 
   // top-k: the k best (no mass rule); top-p: at most Cap
