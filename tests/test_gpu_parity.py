@@ -669,3 +669,30 @@ def test_bounded_wait_gives_up_and_reports():
     mask, out = U.run_fused_step(dc, q, k, v, w.p)
     torch.cuda.synchronize()
     assert dc.read_status()[B.ST_FLAGS] == 0 and torch.isfinite(out).all()
+
+
+@pytest.mark.parametrize("p", [0.5, 0.95])
+def test_long_rows_read_from_global(p):
+    """Rows longer than the top-p kernel's shared-memory score cache (R > 40960): every
+    pass reads the scores from global memory in batches and the mask words are staged
+    for the index pass. One head of 45k candidates and one of 44k (ragged), through
+    the mask-only entry and the fused step, against the oracle."""
+    w = synth.small(batch=2, n_kv_heads=1, n_q_heads=4, context=None, len_range=(44000, 45500),
+                    sparse_cap=48000, dense_window=64, condensed_slots=32, p=p, temp_range=(0.5, 3.0))
+    st = synth.initial_state(w)
+    assert st.R > 40960
+    dc = DecodeCache.from_state(st)
+    dc2 = DecodeCache.from_state(st)
+    (q, k, v), (q_ex, k_ex, v_ex) = U.upload_step(dc, w, st, 0)
+    dc.append(k, v)
+    mask = dc.new_mask()
+    dc.score_calibrate_topp(q, p, mask)
+    mask2, out2 = U.run_fused_step(dc2, q, k, v, p)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, mask2)
+    units = {(b, h): oracle_unit_from_state(st, b, h) for b in range(w.batch)
+             for h in range(w.n_kv_heads)}
+    cmp = U.StepCompare(w.dtype)
+    compare_step(w, st, dc2, mask2, out2, units, q_ex, k_ex, v_ex, p, cmp)
+    assert dc2.read_status()[B.ST_FLAGS] == 0
+    U.record("long_rows", p=p, **cmp.summary())
