@@ -279,7 +279,8 @@ int hardkv_score_topk(const hardkv_desc *desc, const hardkv_cache *cache, const 
  * max-pooled logit: sec. 2.B calibrates "scores" into one probability space, whatever
  * produced them). scores: device float [B,H,R], candidate j of (b,h) (position
  * s_lo + j, j < d_lo - s_lo) at scores[(b*H + h)*R + j], 16-byte aligned; other entries
- * are not read. rule HARDKV_RULE_TOPP: calibrated top-p with tau (device float [B,H] or
+ * do not affect the result (the row is copied in 16-byte units, so up to three entries
+ * past a head's candidates are read). rule HARDKV_RULE_TOPP: calibrated top-p with tau (device float [B,H] or
  * NULL = 1) and 0 < p <= 1, at most Cap kept, exactly as hardkv_score_calibrate_topp
  * after its score stage; HARDKV_RULE_TOPK: the top_k best (1 <= top_k <= Cap; p and
  * tau unused). The head's maximum is taken from the scores themselves. mask as in
