@@ -11,7 +11,9 @@ import os
 import re
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libhardkv.so")
+# HARDKV_CHECKED=1 selects the bounds-checked build (libhardkv_checked.so)
+LIB_PATH = os.path.join(HERE, "libhardkv_checked.so" if os.environ.get("HARDKV_CHECKED") == "1"
+                        else "libhardkv.so")
 HEADER = os.path.join(HERE, "..", "include", "hardkv.h")
 
 OK, EINVAL, EALIGN, EDTYPE, ECAP, ECUDA, ESCRATCH = 0, -1, -2, -3, -4, -5, -6
@@ -24,7 +26,7 @@ CAL_TAU, CAL_ENTROPY = 0, 1
 STATUS_WORDS = 8
 ST_FLAGS, ST_CLAMPS, ST_NEAR_TIES, ST_MERGED, ST_MOVES, ST_SELECTIONS = range(6)
 DEV_RING_OVERFLOW, DEV_BAD_BOUNDS, DEV_SEGMENTS, DEV_WAIT_TIMEOUT = 1, 2, 4, 8
-DEV_SELECT, DEV_POOL_SHORT = 16, 32
+DEV_SELECT, DEV_POOL_SHORT, DEV_CHECK = 16, 32, 64
 PAGE_ROWS = 16
 POOL_FREE, POOL_RETURNED, POOL_CTL_WORDS = 0, 1, 4
 STEP_EVENTS = 6

@@ -74,6 +74,19 @@ __device__ __forceinline__ void flag(uint32_t *status, uint32_t bit) {
   atomicOr(status + HARDKV_ST_FLAGS, bit);
 }
 
+// In-bounds test of an index before an access. The checked build (-DHARDKV_CHECKED)
+// evaluates it and, when it fails, records HARDKV_DEV_CHECK and makes the caller skip
+// the access; the normal build takes every access (the indices are in range by
+// construction, which the checked build verifies on the test workloads).
+#ifdef HARDKV_CHECKED
+__device__ __forceinline__ bool in_bounds(uint32_t *status, bool ok) {
+  if (!ok) flag(status, HARDKV_DEV_CHECK);
+  return ok;
+}
+#else
+__device__ __forceinline__ bool in_bounds(uint32_t *, bool) { return true; }
+#endif
+
 // Head-wise block manager (HARD-KV sec. 2.C "Metadati"). A head that needs `need` blocks
 // keeps its first min(have, need) blocks, returns the surplus to ret_list and takes the
 // deficit from the top of free_list (an atomic decrement reserves a disjoint range; a
@@ -108,8 +121,12 @@ __device__ int pool_assign(const Cache &c, int u, int need, PoolAlloc *pa) {
   __syncthreads();
   const PoolAlloc a = *pa;
   for (int i = threadIdx.x; i < a.have - a.keep; i += blockDim.x)
-    c.ret_list[a.give_at + i] = tab[a.keep + i];
-  for (int i = threadIdx.x; i < a.got; i += blockDim.x) tab[a.keep + i] = c.free_list[a.take_from + i];
+    if (in_bounds(c.status, a.give_at + i < c.pool_blocks && a.keep + i < c.tab_blocks))
+      c.ret_list[a.give_at + i] = tab[a.keep + i];
+  for (int i = threadIdx.x; i < a.got; i += blockDim.x)
+    if (in_bounds(c.status, a.keep + i < c.tab_blocks && a.take_from + i < c.pool_blocks &&
+                               (unsigned)c.free_list[a.take_from + i] < (unsigned long long)c.pool_blocks))
+      tab[a.keep + i] = c.free_list[a.take_from + i];
   __syncthreads();
   const int held = a.keep + a.got;
   if (threadIdx.x == 0) c.blk_cnt[u] = held;
@@ -125,7 +142,8 @@ __device__ void pool_merge(const Cache &c) {
     s_r = c.pool_ctl[HARDKV_POOL_RETURNED];
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < s_r; i += blockDim.x) c.free_list[s_f + i] = c.ret_list[i];
+  for (int i = threadIdx.x; i < s_r; i += blockDim.x)
+    if (in_bounds(c.status, s_f + i < c.pool_blocks)) c.free_list[s_f + i] = c.ret_list[i];
   __syncthreads();
   if (threadIdx.x == 0) {
     c.pool_ctl[HARDKV_POOL_FREE] = s_f + s_r;

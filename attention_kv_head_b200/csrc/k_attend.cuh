@@ -252,6 +252,17 @@ __device__ __forceinline__ bool last_to_finish(const AttendParams &ap, const int
 constexpr uint32_t kRowRing = 1u << 30, kRowCompact = 2u << 30, kRowCond = 3u << 30;
 constexpr uint32_t kRowGather = 1u << 29, kRowIdx = (1u << 29) - 1;
 
+// Rows a row code may address: ring rows < R, compact slots < Cap (pool rows < pool
+// blocks x 16 on the paged tier), Condensed slots < C.
+__device__ __forceinline__ long long compact_rows(const Shape &sh, const Cache &c) {
+  return c.k_pool ? c.pool_blocks * HARDKV_PAGE_ROWS : (long long)sh.cap;
+}
+__device__ __forceinline__ bool code_in_bounds(const Shape &sh, const Cache &c, uint32_t code) {
+  const uint32_t kind = code & (3u << 30), idx = code & kRowIdx;
+  const long long lim = kind == kRowRing ? sh.R : kind == kRowCompact ? compact_rows(sh, c) : sh.C;
+  return in_bounds(c.status, kind == 0u || (long long)idx < lim);
+}
+
 struct UnitView {
   Bounds bd;
   int n_u, nd, wgt;
@@ -451,8 +462,9 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
         const uint8_t *base = kind == kRowRing ? (kv ? vring : kring)
                               : kind == kRowCompact ? (kv ? vsp : ksp)
                                                     : (kv ? vcd : kcd);
-        const uint8_t *src = kind ? base + (size_t)(code & kRowIdx) * rb + ch * 16 : kcd;
-        cp_async16(dst0 + kv * Cfg::TILE_BYTES + r * D * 4 + ch * 16, src, kind ? 16 : 0);
+        const bool live = kind && code_in_bounds(sh, c, code);
+        const uint8_t *src = live ? base + (size_t)(code & kRowIdx) * rb + ch * 16 : kcd;
+        cp_async16(dst0 + kv * Cfg::TILE_BYTES + r * D * 4 + ch * 16, src, live ? 16 : 0);
       }
       cp_async_commit();
     };
@@ -474,8 +486,10 @@ __global__ void __launch_bounds__(kF32Threads) attend_f32_kernel(Shape sh, Cache
       if (v.gather && v.rewrite) {  // Rewrite Cache: kept rows of this tile -> compact slots
         for (int i = tid; i < kAttRows * Cfg::VEC * 2; i += kF32Threads) {
           const int r = i / (2 * Cfg::VEC), kv = (i / Cfg::VEC) & 1, ch = i % Cfg::VEC;
-          if (codes[stg * kAttRows + r] & kRowGather) {
-            uint8_t *dst = (kv ? vsp : ksp) + (size_t)compact_slot_row(v, r0 + t * kAttRows + r) * rb + ch * 16;
+          const size_t slot = compact_slot_row(v, r0 + t * kAttRows + r);
+          if ((codes[stg * kAttRows + r] & kRowGather) &&
+              in_bounds(c.status, (long long)slot < compact_rows(sh, c))) {
+            uint8_t *dst = (kv ? vsp : ksp) + slot * rb + ch * 16;
             *reinterpret_cast<uint4 *>(dst) =
                 *reinterpret_cast<const uint4 *>(kvb + kv * Cfg::TILE_BYTES + r * D * 4 + ch * 16);
           }

@@ -249,6 +249,7 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
     auto src_of = [&](uint32_t code, int kv) -> const uint8_t * {
       const uint32_t kind = code & (3u << 30);
       const size_t off = (size_t)(code & kRowIdx) * rb;
+      if (!code_in_bounds(sh, c, code)) return nullptr;  // checked build only
       if (kind == kRowRing) return (kv ? vring : kring) + off;
       if (kind == kRowCompact) return (kv ? vsp : ksp) + off;
       if (kind == kRowCond) return (kv ? vcd : kcd) + off;
@@ -311,8 +312,10 @@ __global__ void __launch_bounds__(kWsThreads, 3) attend_ws_kernel(Shape sh, Cach
           const int r = lane & 15;
           const size_t slot = compact_slot_row(v, r0 + t * kAttRows + w * kWsRows + r);
           const int kv = lane >> 4;
-          bulk_s2g((kv ? vsp : ksp) + slot * rb, ks + kv * Cfg::SLICE + r * Cfg::STRIDE, (uint32_t)rb);
-          bulk_commit();
+          if (in_bounds(c.status, (long long)slot < compact_rows(sh, c))) {
+            bulk_s2g((kv ? vsp : ksp) + slot * rb, ks + kv * Cfg::SLICE + r * Cfg::STRIDE, (uint32_t)rb);
+            bulk_commit();
+          }
         }
       } else {
         __syncwarp();

@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(ScoreTma<D>::THREADS)
         const long long pos = pbase + g + 8 * hr;
         if (pos >= s_lo && pos < d_lo) {
           const float s = (hr ? v8 : v0) * sh.scale;
-          scores[(size_t)u * sh.R + (size_t)(pos - s_lo)] = s;
+          if (in_bounds(c.status, pos - s_lo < sh.R)) scores[(size_t)u * sh.R + (size_t)(pos - s_lo)] = s;
           tmax = fmaxf(tmax, s);
         }
       }
@@ -365,7 +365,7 @@ __global__ void __launch_bounds__(128)
       }
     }
     const float s = best * sh.scale;
-    if (lane == 0) scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
+    if (lane == 0 && in_bounds(c.status, pos - bd.s_lo < sh.R)) scores[(size_t)u * sh.R + (size_t)(pos - bd.s_lo)] = s;
     tmax = fmaxf(tmax, s);
   }
   if (lane == 0) tile_max[(size_t)u * tm_stride + lt * kPartsPerTile + warp] = tmax;

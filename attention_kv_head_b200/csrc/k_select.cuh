@@ -834,7 +834,8 @@ __global__ void __launch_bounds__(kSelThreads)
       uint32_t mine = 0u;
 #pragma unroll
       for (int k = 0; k < KW; ++k) mine = lane == k ? wb[k] : mine;
-      if (lane < K && warp * K + lane < nwords) mrow[warp * K + lane] = mine;
+      if (lane < K && warp * K + lane < nwords && in_bounds(c.status, warp * K + lane < sh.mask_words))
+        mrow[warp * K + lane] = mine;
     }
     if (WRITE_IDX) {
       if (lane == 0) S.scan[warp] = wcount;
@@ -844,7 +845,8 @@ __global__ void __launch_bounds__(kSelThreads)
       for (int k = 0; k < KW; ++k) {
         const int wi = warp * K + k;
         const int slot = base + __popc(wb[k] & lt_mask);
-        if (((wb[k] >> lane) & 1u) && slot < n) idx[slot] = bd.s_lo + wi * 32 + lane;
+        if (((wb[k] >> lane) & 1u) && slot < n && in_bounds(c.status, slot < sh.cap))
+          idx[slot] = bd.s_lo + wi * 32 + lane;
         base += __popc(wb[k]);
       }
     }
@@ -873,8 +875,10 @@ __global__ void __launch_bounds__(kSelThreads)
         }
         const unsigned word = __ballot_sync(0xffffffffu, kept);
         if (lane == 0) {
-          if (mrow) mrow[wi] = word;
-          wbuf[wi] = word;
+          if (in_bounds(c.status, wi < sh.mask_words && wi < 6 * kBins)) {
+            if (mrow) mrow[wi] = word;
+            wbuf[wi] = word;
+          }
         }
         wcount += __popc(word);
       }
@@ -888,7 +892,8 @@ __global__ void __launch_bounds__(kSelThreads)
         if (wi >= nwords) break;
         const unsigned word = wbuf[wi];
         const int slot = base + __popc(word & lt_mask);
-        if (((word >> lane) & 1u) && slot < n) idx[slot] = bd.s_lo + wi * 32 + lane;
+        if (((word >> lane) & 1u) && slot < n && in_bounds(c.status, slot < sh.cap))
+          idx[slot] = bd.s_lo + wi * 32 + lane;
         base += __popc(word);
       }
     }
@@ -997,6 +1002,10 @@ __global__ void __launch_bounds__(kSelThreads)
     const int pos = list_pos[e2];
     const size_t src_row = (size_t)(pos % sh.R) * sh.d,
                  dst_row = compact_row(c, sh.cap, u, slot) * sh.d;
+    if (!in_bounds(c.status, (long long)(dst_row / sh.d) <
+                                 (c.k_pool ? c.pool_blocks * HARDKV_PAGE_ROWS
+                                           : (long long)(sh.B * sh.H) * sh.cap)))
+      continue;
     if (kv == 0) {
       reinterpret_cast<uint4 *>(ks + dst_row)[v2] = reinterpret_cast<const uint4 *>(kr + src_row)[v2];
       if (v2 == 0) idx[slot] = pos;
@@ -1033,7 +1042,8 @@ __global__ void __launch_bounds__(256) flatten_sum_kernel(Shape sh, Cache c, int
     if (u == U - 1) offsets[U] = base + n;
   }
   const int32_t *idx = c.sp_idx + (size_t)u * sh.cap;
-  for (int j = tid; j < n; j += 256) flat[base + j] = idx[j];
+  for (int j = tid; j < n; j += 256)
+    if (in_bounds(c.status, (long long)base + j < (long long)U * sh.cap)) flat[base + j] = idx[j];
 }
 
 }  // namespace hardkv

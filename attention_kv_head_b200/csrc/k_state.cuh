@@ -227,6 +227,7 @@ __global__ void __launch_bounds__(kCondenseThreads) condense_kernel(Shape sh, Ca
     __syncthreads();
     const int sstar = red_i[NW];
     if (sstar == 0x7fffffff) break;  // no mergeable slot: nothing to merge into
+    if (!in_bounds(c.status, sstar >= 0 && sstar < C)) break;  // checked build only
     const double wd = (double)w[sstar];
     for (int ch = tid; ch < d; ch += kCondenseThreads) {
       double kk = __dadd_rn(__dmul_rn(wd, (double)to_f32(kcd[(size_t)sstar * d + ch])),

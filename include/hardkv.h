@@ -122,6 +122,8 @@ enum {
 #define HARDKV_DEV_SELECT       16u  /* top-p found no cut (inconsistent input): unit kept all */
 #define HARDKV_DEV_POOL_SHORT   32u  /* paged compact tier: a rewritten selection got fewer
                                         blocks than it needed and kept its first rows only */
+#define HARDKV_DEV_CHECK        64u  /* bounds-checked build (libhardkv_checked.so) only: an
+                                        index was out of range; that access was skipped */
 
 /* Rows per block of the paged compact tier (hardkv_cache::k_pool). */
 #define HARDKV_PAGE_ROWS 16
