@@ -320,6 +320,7 @@ def run_gpu(args, world, rank, local) -> dict:
 
     # algorithmic bytes of every step of the window, from the device state after it
     per_step = []
+    pool_held = 0   # paged tier: most blocks the heads held after any step of the window
     with torch.cuda.stream(stream):
         for row in evs + [ends]:
             for e_ in row:
@@ -334,6 +335,8 @@ def run_gpu(args, world, rank, local) -> dict:
             cur["live"] = ((cur["sp_idx"] >= cur["s_lo"][:, None, None]) &
                            (np.arange(w.sparse_cap)[None, None, :] < cur["n_kept"][:, :, None])).sum(-1)
             per_step.append(step_bytes(w, cur))
+            if dc.blk_cnt is not None:
+                pool_held = max(pool_held, int(dc.blk_cnt.sum().item()))
         by = sum_bytes(per_step)
         for _ in range(2):                         # eager warm-up (sets kernel attributes)
             restore()
@@ -414,7 +417,11 @@ def run_gpu(args, world, rank, local) -> dict:
                 clocks=clk.summary(), e2e_ms=e2e_mean, kernels_per_step=kernels_per_step,
                 h2d=int(q.numel() * q.element_size() + 2 * k.numel() * k.element_size()),
                 d2h=int(out.numel() * 4), status=status, p50_ms=float(np.median(win_ms)) / N,
-                select=sel)
+                select=sel, pool=None if pool is None else dict(
+                    pool_blocks=int(pool), blocks_held_max=pool_held,
+                    bytes_held_max=pool_held * Bn.PAGE_ROWS * w.head_dim * dc.k_pool.element_size() * 2,
+                    contiguous_bytes=w.batch * w.n_kv_heads * w.sparse_cap * w.head_dim *
+                    dc.k_pool.element_size() * 2))
 
 
 # ----------------------------------------------------------------------------- oracle
@@ -635,6 +642,7 @@ def main(argv=None):
         "gpu_launches": r["kernels_per_step"] * args.steps * N,
         "clocks": r["clocks"],
         "device_status": [int(x) for x in r["status"]],
+        **({"compact_tier_memory": r["pool"]} if r.get("pool") else {}),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = oracle_timing(w, args.oracle_seconds)
