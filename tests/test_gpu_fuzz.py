@@ -2,10 +2,13 @@
 
 Each case draws the shapes (dtype, head_dim, KV heads, GQA group, batch, Dense window,
 block, Condensed slots, sinks, Sparse capacity, fixed or ragged lengths), the
-selection rule (calibrated top-p at p from 0.5 to 1, or fixed top-k), the layout
-(Rewrite Cache, Sparse Loading, or the MTI rule with random thresholds), the compact
-tier (contiguous or a paged pool), the condense mode and the reselection cadence, and
-runs several steps with the oracle following every unit. Bars as in the other parity
+selection rule (calibrated top-p at p from 0.5 to 1, or fixed top-k), the calibration
+of top-p (tau = 1, caller temperatures on both sides of 1, or the entropy-matched
+temperature), the layout (Rewrite Cache, Sparse Loading, or the MTI rule with random
+thresholds), the compact tier (contiguous or a paged pool), the condense mode and the
+reselection cadence, and runs several steps with the oracle following every unit.
+Under the entropy-matched calibration the oracle selects at the GPU's temperature, and
+that temperature must match the oracle's own solve within 1e-4 (relative). Bars as in the other parity
 tests: boundaries, kept counts and indices bit-exact (on the GPU's accepted mask),
 masks within the near-threshold rule (top-k: within the score rounding of the k-th
 score), the layout decision equal to the oracle's MTI rule, attention within the
@@ -27,7 +30,7 @@ pytestmark = pytest.mark.gpu
 if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
-N_CASES = 64
+N_CASES = 256
 
 
 def draw(seed: int):
@@ -60,7 +63,10 @@ def draw(seed: int):
     mti = (lo, int(lo + r.randint(0, 400)), float(np.float32(r.choice([0.05, 0.5, 2.0]))))
     select = ["all", "moved"][r.randint(2)]
     paged = bool(r.rand() < 0.5)
-    return w, rule, k, layout, mti, select, paged
+    # drawn from a stream of its own, so the draws above stay what they were
+    cal = "tau1" if rule == "topk" else \
+        ["tau1", "tau", "entropy"][np.random.RandomState(5000 + seed).choice(3, p=[0.4, 0.3, 0.3])]
+    return w, rule, k, layout, mti, select, paged, cal
 
 
 def pool_partition(dc: DecodeCache):
@@ -74,7 +80,7 @@ def pool_partition(dc: DecodeCache):
 
 @pytest.mark.parametrize("seed", range(N_CASES))
 def test_random_configuration(seed):
-    w, rule, k, layout, (l_lo, l_hi, surcharge), select, paged = draw(seed)
+    w, rule, k, layout, (l_lo, l_hi, surcharge), select, paged, cal = draw(seed)
     st = synth.initial_state(w)
     pool = w.batch * w.n_kv_heads * (-(-w.sparse_cap // B.PAGE_ROWS)) if paged else None
     dc = DecodeCache.from_state(st, pool_blocks=pool)
@@ -83,6 +89,13 @@ def test_random_configuration(seed):
     mode = {"rewrite": B.LAYOUT_REWRITE, "sparse": B.LAYOUT_SPARSE_LOAD, "mti": B.LAYOUT_MTI}[layout]
     pol = B.LayoutPolicy(mode, -1, l_lo, l_hi, surcharge)
     sel_kw = dict(rule=B.RULE_TOPK, top_k=min(k, w.sparse_cap)) if rule == "topk" else {}
+    tau_np = synth.calibration_taus(w) if cal == "tau" else None
+    tau_dev = None if tau_np is None else torch.from_numpy(tau_np).to(dc.device)
+    tau_out = None
+    if cal == "entropy":
+        tau_out = torch.zeros(w.batch, w.n_kv_heads, dtype=torch.float32, device=dc.device)
+        sel_kw = dict(calibration=B.CAL_ENTROPY, tau_out=tau_out)
+    worst_tau = 0.0
     cmp = U.StepCompare(w.dtype)
     G = w.group
     diverged = set()
@@ -91,9 +104,10 @@ def test_random_configuration(seed):
         rs = "all" if (t == 0 or select == "all") else "moved"
         mask = dc.new_mask()
         out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
-        dc.step(q, kn, vn, out, w.p, mask=mask, layout=pol,
+        dc.step(q, kn, vn, out, w.p, tau=tau_dev, mask=mask, layout=pol,
                 select_mode=B.SELECT_ALL if rs == "all" else B.SELECT_MOVED, **sel_kw)
         torch.cuda.synchronize()
+        taus = None if tau_out is None else tau_out.cpu().numpy()
         m = mask.cpu().numpy().view(np.uint32)
         n_kept, sp_idx, sp_mode = (dc.n_kept.cpu().numpy(), dc.sp_idx.cpu().numpy(),
                                    dc.sp_mode.cpu().numpy())
@@ -104,8 +118,14 @@ def test_random_configuration(seed):
             if (b, h) in diverged:
                 continue
             qg = q_ex[b, h * G:(h + 1) * G]
-            res = un.step(qg, k_ex[b, h], v_ex[b, h], 1.0, w.p, reselect=rs, rule=rule,
+            tau_u = float(taus[b, h]) if taus is not None else U.tau_of(tau_np, b, h)
+            res = un.step(qg, k_ex[b, h], v_ex[b, h], tau_u, w.p, reselect=rs, rule=rule,
                           k=min(k, w.sparse_cap))
+            if cal == "entropy" and res.sel is not None and un.d_lo - un.s_lo > 1:
+                Ks = un.K[un.s_lo:un.d_lo]
+                tau_or = O.entropy_matched_tau(O.score(qg, Ks), O.attention_entropy(qg, Ks))
+                worst_tau = max(worst_tau, abs(tau_u / tau_or - 1.0))
+                assert worst_tau <= 1e-4, (seed, t, b, h, tau_u, tau_or)
             assert (bounds[0][b], bounds[1][b], bounds[2][b]) == (un.len, un.d_lo, un.s_lo)
             if res.merge is not None and res.merge.gaps and min(res.merge.gaps) <= U.MERGE_TIE:
                 diverged.add((b, h))
@@ -142,5 +162,6 @@ def test_random_configuration(seed):
             pool_partition(dc)
     assert dc.read_status()[B.ST_FLAGS] == 0
     assert len(diverged) <= max(1, len(units) // 4)
-    U.record("fuzz", seed=seed, rule=rule, layout=layout, select=select, paged=paged,
-             dtype=w.dtype, units=len(units), steps=w.steps, diverged=len(diverged), **cmp.summary())
+    U.record("fuzz", seed=seed, rule=rule, calibration=cal, layout=layout, select=select,
+             paged=paged, dtype=w.dtype, units=len(units), steps=w.steps, diverged=len(diverged),
+             worst_tau_rel=worst_tau, **cmp.summary())
