@@ -1,19 +1,19 @@
 """Seeded random configurations of the fused decode step against the oracle.
 
-Each case draws the shapes (dtype, head_dim, KV heads, GQA group, batch, Dense window,
-block, Condensed slots, sinks, Sparse capacity, fixed or ragged lengths), the
+Each case draws the shapes (dtype, head_dim, KV heads, GQA group 1-16, batch, Dense
+window, block, Condensed slots, sinks, Sparse capacity, fixed or ragged lengths), the
 selection rule (calibrated top-p at p from 0.5 to 1, or fixed top-k), the calibration
 of top-p (tau = 1, caller temperatures on both sides of 1, or the entropy-matched
 temperature), the layout (Rewrite Cache, Sparse Loading, or the MTI rule with random
 thresholds), the compact tier (contiguous or a paged pool), the condense mode and the
 reselection cadence, and runs several steps with the oracle following every unit.
 Under the entropy-matched calibration the oracle selects at the GPU's temperature, and
-that temperature must match the oracle's own solve within 1e-4 (relative). Bars as in the other parity
-tests: boundaries, kept counts and indices bit-exact (on the GPU's accepted mask),
-masks within the near-threshold rule (top-k: within the score rounding of the k-th
-score), the layout decision equal to the oracle's MTI rule, attention within the
-dtype's tolerance, Condensed state bit-exact except after merge near-ties, the pool a
-partition of its blocks.
+that temperature must match the oracle's own solve within 1e-4 (relative). Bars as in
+the other parity tests: boundaries, kept counts and indices bit-exact (on the GPU's
+accepted mask), masks within the near-threshold rule (top-k: within the score rounding
+of the k-th score), the layout decision equal to the oracle's MTI rule, attention
+within the dtype's tolerance, Condensed state bit-exact except after merge near-ties,
+the pool a partition of its blocks.
 """
 import numpy as np
 import pytest
@@ -35,10 +35,18 @@ N_CASES = 256
 
 def draw(seed: int):
     r = np.random.RandomState(1000 + seed)
+    # a second stream for the calibration and the wide groups, so the draws from `r`
+    # stay what they were before those were added
+    r2 = np.random.RandomState(5000 + seed)
+    cal_pick = ["tau1", "tau", "entropy"][r2.choice(3, p=[0.4, 0.3, 0.3])]
+    wide = r2.rand() < 0.12   # G = 12 or 16: two query tiles of 8 in the kernels
+    G_wide = int([12, 16][r2.randint(2)])
     dtype = [synth.BF16, synth.F32][r.randint(2)]
     d = [64, 128][r.randint(2)]
     H = int(r.randint(1, 4))
     G = int([1, 2, 4, 5, 8][r.randint(5)])
+    if wide:
+        G = G_wide
     Bn = int(r.randint(1, 5))
     W = int([16, 32, 48, 64][r.randint(4)])
     blk = int([8, 16][r.randint(2)])
@@ -63,9 +71,7 @@ def draw(seed: int):
     mti = (lo, int(lo + r.randint(0, 400)), float(np.float32(r.choice([0.05, 0.5, 2.0]))))
     select = ["all", "moved"][r.randint(2)]
     paged = bool(r.rand() < 0.5)
-    # drawn from a stream of its own, so the draws above stay what they were
-    cal = "tau1" if rule == "topk" else \
-        ["tau1", "tau", "entropy"][np.random.RandomState(5000 + seed).choice(3, p=[0.4, 0.3, 0.3])]
+    cal = "tau1" if rule == "topk" else cal_pick
     return w, rule, k, layout, mti, select, paged, cal
 
 
