@@ -1,12 +1,14 @@
-"""Seeded random configurations of the fused decode step against the oracle.
+"""Seeded random configurations of the decode step against the oracle.
 
 Each case draws the shapes (dtype, head_dim, KV heads, GQA group 1-16, batch, Dense
 window, block, Condensed slots, sinks, Sparse capacity, fixed or ragged lengths), the
 selection rule (calibrated top-p at p from 0.5 to 1, or fixed top-k), the calibration
 of top-p (tau = 1, caller temperatures on both sides of 1, or the entropy-matched
 temperature), the layout (Rewrite Cache, Sparse Loading, or the MTI rule with random
-thresholds), the compact tier (contiguous or a paged pool), the condense mode and the
-reselection cadence, and runs several steps with the oracle following every unit.
+thresholds), the compact tier (contiguous or a paged pool), the condense mode, the
+reselection cadence and the entry points (the fused step, or in a quarter of the cases
+its standalone calls: append, condense, selection, regularization under the layout
+policy, attention), and runs several steps with the oracle following every unit.
 Under the entropy-matched calibration the oracle selects at the GPU's temperature, and
 that temperature must match the oracle's own solve within 1e-4 (relative). Bars as in
 the other parity tests: boundaries, kept counts and indices bit-exact (on the GPU's
@@ -41,6 +43,9 @@ def draw(seed: int):
     cal_pick = ["tau1", "tau", "entropy"][r2.choice(3, p=[0.4, 0.3, 0.3])]
     wide = r2.rand() < 0.12   # G = 12 or 16: two query tiles of 8 in the kernels
     G_wide = int([12, 16][r2.randint(2)])
+    # the fused step, or the same step as its standalone calls (append, condense,
+    # selection, regularization with the layout policy, attention)
+    path = "unfused" if r2.rand() < 0.25 else "fused"
     dtype = [synth.BF16, synth.F32][r.randint(2)]
     d = [64, 128][r.randint(2)]
     H = int(r.randint(1, 4))
@@ -72,7 +77,7 @@ def draw(seed: int):
     select = ["all", "moved"][r.randint(2)]
     paged = bool(r.rand() < 0.5)
     cal = "tau1" if rule == "topk" else cal_pick
-    return w, rule, k, layout, mti, select, paged, cal
+    return w, rule, k, layout, mti, select, paged, cal, path
 
 
 def pool_partition(dc: DecodeCache):
@@ -86,7 +91,7 @@ def pool_partition(dc: DecodeCache):
 
 @pytest.mark.parametrize("seed", range(N_CASES))
 def test_random_configuration(seed):
-    w, rule, k, layout, (l_lo, l_hi, surcharge), select, paged, cal = draw(seed)
+    w, rule, k, layout, (l_lo, l_hi, surcharge), select, paged, cal, path = draw(seed)
     st = synth.initial_state(w)
     pool = w.batch * w.n_kv_heads * (-(-w.sparse_cap // B.PAGE_ROWS)) if paged else None
     dc = DecodeCache.from_state(st, pool_blocks=pool)
@@ -110,8 +115,21 @@ def test_random_configuration(seed):
         rs = "all" if (t == 0 or select == "all") else "moved"
         mask = dc.new_mask()
         out = torch.empty(w.batch, w.n_q_heads, w.head_dim, dtype=torch.float32, device=dc.device)
-        dc.step(q, kn, vn, out, w.p, tau=tau_dev, mask=mask, layout=pol,
-                select_mode=B.SELECT_ALL if rs == "all" else B.SELECT_MOVED, **sel_kw)
+        smode = B.SELECT_ALL if rs == "all" else B.SELECT_MOVED
+        if path == "fused":
+            dc.step(q, kn, vn, out, w.p, tau=tau_dev, mask=mask, layout=pol, select_mode=smode,
+                    **sel_kw)
+        else:
+            dc.append(kn, vn)
+            dc.condense()
+            if rule == "topk":
+                dc.score_topk(q, min(k, w.sparse_cap), mask, select_mode=smode)
+            elif cal == "entropy":
+                dc.score_calibrate_entropy_topp(q, w.p, mask, tau_out=tau_out, select_mode=smode)
+            else:
+                dc.score_calibrate_topp(q, w.p, mask, tau=tau_dev, select_mode=smode)
+            dc.regularize(mask, select_mode=smode, layout=pol)
+            dc.decode_attn(q, out)
         torch.cuda.synchronize()
         taus = None if tau_out is None else tau_out.cpu().numpy()
         m = mask.cpu().numpy().view(np.uint32)
@@ -168,6 +186,6 @@ def test_random_configuration(seed):
             pool_partition(dc)
     assert dc.read_status()[B.ST_FLAGS] == 0
     assert len(diverged) <= max(1, len(units) // 4)
-    U.record("fuzz", seed=seed, rule=rule, calibration=cal, layout=layout, select=select,
+    U.record("fuzz", seed=seed, path=path, rule=rule, calibration=cal, layout=layout, select=select,
              paged=paged, dtype=w.dtype, units=len(units), steps=w.steps, diverged=len(diverged),
              worst_tau_rel=worst_tau, **cmp.summary())
