@@ -8,7 +8,8 @@ temperature), the layout (Rewrite Cache, Sparse Loading, or the MTI rule with ra
 thresholds), the compact tier (contiguous or a paged pool), the condense mode, the
 reselection cadence and the entry points (the fused step, or in a quarter of the cases
 its standalone calls: append, condense, selection, regularization under the layout
-policy, attention), and runs several steps with the oracle following every unit.
+policy, attention; some fused cases through the host-buffer entry point, pinned or
+pageable), and runs several steps with the oracle following every unit.
 Under the entropy-matched calibration the oracle selects at the GPU's temperature, and
 that temperature must match the oracle's own solve within 1e-4 (relative). Bars as in
 the other parity tests: boundaries, kept counts and indices bit-exact (on the GPU's
@@ -46,6 +47,9 @@ def draw(seed: int):
     # the fused step, or the same step as its standalone calls (append, condense,
     # selection, regularization with the layout policy, attention)
     path = "unfused" if r2.rand() < 0.25 else "fused"
+    # some fused cases through the host-buffer entry point, pinned or pageable
+    if r2.rand() < 0.2 and path == "fused":
+        path = "host_pinned" if r2.rand() < 0.5 else "host_pageable"
     dtype = [synth.BF16, synth.F32][r.randint(2)]
     d = [64, 128][r.randint(2)]
     H = int(r.randint(1, 4))
@@ -119,6 +123,13 @@ def test_random_configuration(seed):
         if path == "fused":
             dc.step(q, kn, vn, out, w.p, tau=tau_dev, mask=mask, layout=pol, select_mode=smode,
                     **sel_kw)
+        elif path.startswith("host"):
+            host = [t_.cpu() for t_ in (q, kn, vn)] + [torch.full(out.shape, float("nan"))]
+            if path == "host_pinned":
+                host = [t_.pin_memory() for t_ in host]
+            qh, kh, vh, out = host
+            dc.step_host(qh, kh, vh, out, w.p, tau=None if tau_np is None else torch.from_numpy(tau_np),
+                         mask=mask, layout=pol, select_mode=smode, **sel_kw)
         else:
             dc.append(kn, vn)
             dc.condense()
