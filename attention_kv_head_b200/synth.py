@@ -192,6 +192,10 @@ WORKLOADS: dict[str, Workload] = {
     "stress64k": Workload("stress64k", 16, 40, 8, 128, BF16, 65536, None, 512, 1024, 16,
                           9840, 0.95, 128, 1, MERGE, "loguniform", (0.25, 8.0),
                           spike_frac=0.1),
+    # A profiling case for the weighted merge: llama8b_8k's heads with contbatch's 512
+    # Condensed slots, context 2048, MERGE; step 16 moves a block in every sequence.
+    "merge_c512": Workload("merge_c512", 8, 32, 8, 128, BF16, 2048, None, 256, 512, 16,
+                           1280, 0.9, 17, 1, MERGE, "loguniform", (0.5, 4.0)),
 }
 
 

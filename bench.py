@@ -41,9 +41,11 @@ METRIC = "compressed-KV decode tokens/s at batch×ctx; HBM GB/s as % of B200 pea
 L2_BYTES = 126 * 1024 * 1024
 NOMINAL_HBM_GBS = 8000.0
 STAGES = ("append", "condense", "score", "topp", "attend")
+# --path unfused: the step as its standalone calls; "select" is one call (score + top-p)
+UNFUSED_STAGES = ("append", "condense", "select", "regularize", "attend")
 KERNEL_OF_STAGE = {"append": "append_kernel", "condense": "condense_kernel",
                    "score": "score_tma_kernel", "topp": "topp_kernel",
-                   "attend": "attend_ws_kernel"}
+                   "regularize": "compact_kernel", "attend": "attend_ws_kernel"}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -65,15 +67,17 @@ def csrc_digest() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu capture of the current sources."""
+def ncu_traffic(kernel: str, workload: str, path: str = "fused"):
+    """DRAM bytes per launch from a committed ncu capture of the current sources (of the
+    same workload and the same path: fused step or standalone calls)."""
     p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     if not os.path.exists(p):
         return None
     try:
         d = json.load(open(p))
         e = d.get(kernel)
-        if e and e.get("csrc_sha") == csrc_digest() and e.get("workload") == workload:
+        if (e and e.get("csrc_sha") == csrc_digest() and e.get("workload") == workload
+                and e.get("path", "fused") == path):
             return float(e["dram_bytes_per_launch"])
     except Exception:
         return None
@@ -167,11 +171,12 @@ def job_tokens_per_s(world: int, batch: int, max_step_ms: float) -> float:
 
 # ----------------------------------------------------------------------------- bytes
 
-def step_bytes(w, st: dict) -> dict:
+def step_bytes(w, st: dict, fused: bool = True) -> dict:
     """Bytes one decode step must move (reads + writes), per stage, from the device state
     after the step: `st` holds len / d_lo / s_lo / moved [B], n_kept / sp_mode [B,H],
     live [B,H] (kept rows whose position is still Sparse) and `reselect` [B] (sequences
-    that scored and selected in this step).
+    that scored and selected in this step). fused = False: the step as its standalone
+    calls (stages append, condense, select, regularize, attend; unfused_bytes).
 
       append    k_new, v_new read; their ring rows written
       condense  per unit of a moved sequence (MERGE): the block's K/V and the C slots'
@@ -184,6 +189,8 @@ def step_bytes(w, st: dict) -> dict:
                 written to the compact layout in a reselecting step; otherwise read from
                 the compact layout or the ring), their index, the Dense and Condensed
                 rows, the Condensed weights, q and the fp32 output"""
+    if not fused:
+        return unfused_bytes(w, st)
     e = 2 if w.dtype == "bf16" else 4
     d, H, G, C = w.head_dim, w.n_kv_heads, w.group, w.condensed_slots
     row = 2 * d * e                                             # one K row + one V row
@@ -218,8 +225,46 @@ def step_bytes(w, st: dict) -> dict:
     return by
 
 
+def unfused_bytes(w, st: dict) -> dict:
+    """step_bytes of the step as its standalone calls: the selection writes only the mask
+    (the index comes from the compaction), the compaction reads each reselecting unit's
+    mask and writes its Cap-long index and, under Rewrite Cache, reads its kept rows
+    from the ring and writes them to the compact layout, and the attention then reads
+    every kept row once (compact rows, or ring rows through the index)."""
+    e = 2 if w.dtype == "bf16" else 4
+    d, H, G, C = w.head_dim, w.n_kv_heads, w.group, w.condensed_slots
+    row = 2 * d * e
+    Ls = (st["d_lo"] - st["s_lo"]).astype(np.int64)
+    dense = (st["len"] - st["d_lo"]).astype(np.int64)
+    resel = st["reselect"].astype(bool)
+    moved = st["moved"].astype(bool)
+    n = st["n_kept"].astype(np.int64)
+    live = st["live"].astype(np.int64)
+    rw = st["sp_mode"].astype(bool)
+    U = w.batch * H
+    Lsel = int(Ls[resel].sum()) * H
+    words = int(((Ls[resel] + 31) // 32).sum()) * H * 4
+    kept_sel = int(n[resel].sum())
+    rewritten = int((n * (resel[:, None] & rw)).sum())
+    by = {
+        "append": 2 * U * d * e * 2,
+        "condense": (int(moved.sum()) * H * (w.block + 2 * C) * row
+                     if w.condense_mode == 1 else 0),
+        "select": Lsel * d * e + int(resel.sum()) * H * G * d * e + Lsel * 4   # score
+                  + Lsel * 4 + words,                                            # top-p
+        "regularize": words + int(resel.sum()) * H * w.sparse_cap * 4 + 2 * rewritten * row,
+        "attend": (kept_sel + int((live * ~resel[:, None]).sum())) * row + int(n.sum()) * 4
+                  + (int(dense.sum()) * H + U * C) * row + U * C * 4
+                  + w.batch * w.n_q_heads * d * e + w.batch * w.n_q_heads * d * 4,
+    }
+    by["total"] = sum(by.values())
+    by["sum_kept"] = kept_sel
+    by["kept_fraction"] = kept_sel / max(Lsel, 1)
+    return by
+
+
 def sum_bytes(per_step: list) -> dict:
-    keys = ("append", "condense", "score", "topp", "attend", "total", "sum_kept")
+    keys = [k for k in per_step[0] if k != "kept_fraction"]
     out = {k: sum(b[k] for b in per_step) for k in keys}
     sel_L = sum(b["sum_kept"] / b["kept_fraction"] for b in per_step if b["kept_fraction"] > 0)
     out["kept_fraction"] = out["sum_kept"] / sel_L if sel_L else 0.0
@@ -305,18 +350,54 @@ def run_gpu(args, world, rank, local) -> dict:
         flush.zero_()                      # write 2 x L2 ...
         flush.view(torch.int32).sum()      # ... then read it back: clean lines only
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(Bn.STEP_EVENTS)] for _ in range(N)]
+    # external: recorded during graph capture (by the library, or by unfused_step) they
+    # become event-record nodes that keep their timestamps
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(Bn.STEP_EVENTS)]
+           for _ in range(N)]
     # the timed graph records one event before the window's first kernel and one after
     # its last (graph-launch latency stays outside the timed region)
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ends = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
     edge = [[ends[0] if (t == 0 and i == 0) else
              ends[1] if (t == N - 1 and i == Bn.STEP_EVENTS - 1) else None
              for i in range(Bn.STEP_EVENTS)] for t in range(N)]
 
+    fused = args.path == "fused"
+    stages = STAGES if fused else UNFUSED_STAGES
+
+    def select_call(q):
+        """The selection as one standalone call (score + calibration + top-p or top-k)."""
+        if "top_k" in sel:
+            dc.score_topk(q, sel["top_k"], mask, select_mode=mode, stream=stream)
+        elif sel.get("calibration") == Bn.CAL_ENTROPY:
+            dc.score_calibrate_entropy_topp(q, p, mask, select_mode=mode, stream=stream)
+        else:
+            dc.score_calibrate_topp(q, p, mask, select_mode=mode, stream=stream)
+
+    def unfused_step(q, k, v, ev):
+        """One decode step as the standalone calls; ev[i] (or None) recorded before call i
+        and ev[5] after the last, like the fused step's stage events."""
+        def rec(i):
+            if ev is not None and ev[i] is not None:
+                ev[i].record(stream)
+        rec(0)
+        dc.append(k, v, stream=stream)
+        rec(1)
+        dc.condense(stream=stream)
+        rec(2)
+        select_call(q)
+        rec(3)
+        dc.regularize(mask, select_mode=mode, stream=stream, layout=sel.get("layout"))
+        rec(4)
+        dc.decode_attn(q, out, stream=stream)
+        rec(5)
+
     def window(events=None):
         for t, (q, k, v) in enumerate(inputs):
-            dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream,
-                    events=events[t] if events else None, **sel)
+            if fused:
+                dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream,
+                        events=events[t] if events else None, **sel)
+            else:
+                unfused_step(q, k, v, events[t] if events else None)
 
     # algorithmic bytes of every step of the window, from the device state after it
     per_step = []
@@ -327,14 +408,17 @@ def run_gpu(args, world, rank, local) -> dict:
                 e_.record(stream)                  # create the CUDA events
         restore()
         for t, (q, k, v) in enumerate(inputs):
-            dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream, **sel)
+            if fused:
+                dc.step(q, k, v, out, p, mask=mask, select_mode=mode, stream=stream, **sel)
+            else:
+                unfused_step(q, k, v, None)
             stream.synchronize()
             cur = {n_: getattr(dc, n_).cpu().numpy() for n_ in ("len", "d_lo", "s_lo", "moved", "n_kept",
                                                                "sp_mode", "sp_idx")}
             cur["reselect"] = cur["moved"] if on_move else np.ones(w.batch, bool)
             cur["live"] = ((cur["sp_idx"] >= cur["s_lo"][:, None, None]) &
                            (np.arange(w.sparse_cap)[None, None, :] < cur["n_kept"][:, :, None])).sum(-1)
-            per_step.append(step_bytes(w, cur))
+            per_step.append(step_bytes(w, cur, fused=fused))
             if dc.blk_cnt is not None:
                 pool_held = max(pool_held, int(dc.blk_cnt.sum().item()))
         by = sum_bytes(per_step)
@@ -354,6 +438,8 @@ def run_gpu(args, world, rank, local) -> dict:
     with torch.cuda.graph(gp, stream=stream):
         window(events=evs)
     kernels_per_step = 4 + (1 if w.condense_mode == synth.MERGE else 0)
+    if not fused:   # + the compaction (and, on the paged tier, the pool merge and allocation)
+        kernels_per_step += 1 + (2 if args.paged else 0)
 
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
@@ -384,12 +470,12 @@ def run_gpu(args, world, rank, local) -> dict:
         for _ in range(args.steps):  # stage durations from the event-node replay
             one(gp)
             stage_ms.append([sum(evs[t][i].elapsed_time(evs[t][i + 1]) for t in range(N))
-                             for i in range(len(STAGES))])
+                             for i in range(len(stages))])
     torch.cuda.synchronize()
     dist_barrier(world)
     mean_ms = float(np.mean(win_ms)) / N              # per decode step
     max_ms = dist_max(mean_ms, world, dev)
-    stage_mean = {s: float(np.mean([x[i] for x in stage_ms])) / N for i, s in enumerate(STAGES)}
+    stage_mean = {s: float(np.mean([x[i] for x in stage_ms])) / N for i, s in enumerate(stages)}
 
     # e2e through the host-buffer entry point (every step's inputs copied in, output out)
     host_in = [tuple(t.cpu().pin_memory() for t in x) for x in inputs]
@@ -402,8 +488,17 @@ def run_gpu(args, world, rank, local) -> dict:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for (qh, kh, vh) in host_in:
-                dc.step_host(qh, kh, vh, oh, p, mask=mask, select_mode=mode, stream=stream, **sel)
+            for t, (qh, kh, vh) in enumerate(host_in):
+                if fused:
+                    dc.step_host(qh, kh, vh, oh, p, mask=mask, select_mode=mode, stream=stream,
+                                 **sel)
+                else:   # the standalone calls take device buffers: copies in, output out
+                    q, k, v = inputs[t]
+                    q.copy_(qh, non_blocking=True)
+                    k.copy_(kh, non_blocking=True)
+                    v.copy_(vh, non_blocking=True)
+                    unfused_step(q, k, v, None)
+                    oh.copy_(out, non_blocking=True)
             e1.record(stream)
         stream.synchronize()
         if i >= args.warmup:
@@ -544,6 +639,9 @@ def main(argv=None):
     ap.add_argument("--layout", default="rewrite", choices=["rewrite", "sparse", "mti"])
     ap.add_argument("--paged", action="store_true",
                     help="compact rows in the paged tier (block pool + per-head tables)")
+    ap.add_argument("--path", default="fused", choices=["fused", "unfused"],
+                    help="the fused step (hardkv_decode_step), or the same step as its "
+                         "standalone calls: append, condense, selection, regularize, attention")
     ap.add_argument("--l-lower", type=int, default=64)
     ap.add_argument("--l-upper", type=int, default=1 << 30)
     ap.add_argument("--gather-surcharge", type=float, default=0.5)
@@ -563,6 +661,7 @@ def main(argv=None):
               "selection": args.rule + ("" if args.rule == "topp" else f" k={args.top_k or 'auto'}"),
               "calibration": args.calibration, "layout": args.layout,
               "compact_tier": "paged (16-row blocks)" if args.paged else "contiguous",
+              "path": "fused step" if args.path == "fused" else "standalone calls",
               "l2": "flushed before every timed step: 2 x L2 written, then read back",
               "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
@@ -606,10 +705,12 @@ def main(argv=None):
     if r["select"].get("top_k"):
         config["selection"] = f"topk k={r['select']['top_k']}"
     # dominant kernel by time (per decode step)
-    dom = max(("score", "topp", "attend"), key=lambda s: r["stages"][s])
+    stages = STAGES if args.path == "fused" else UNFUSED_STAGES
+    dom = max(("score", "topp", "attend") if args.path == "fused" else ("regularize", "attend"),
+              key=lambda s: r["stages"][s])
     dom_us = r["stages"][dom] * 1e3
     achieved = by[dom] / (dom_us * 1e-6) / 1e9
-    traffic = ncu_traffic(KERNEL_OF_STAGE[dom], w.name)
+    traffic = ncu_traffic(KERNEL_OF_STAGE[dom], w.name, args.path)
     step_gbs = by["total"] / (r["mean_ms"] * 1e-3) / 1e9
     value = job_tokens_per_s(world, w.batch, r["max_ms"])
     line = {
@@ -619,7 +720,9 @@ def main(argv=None):
         if w.dtype == "bf16" else "f32", "data": "synthetic", "config": config,
         "e2e": {"value": job_tokens_per_s(world, w.batch, r["e2e_ms"]), "unit": "tokens/s",
                 "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "ms_per_step": r["e2e_ms"], "api": "hardkv_decode_step_host"},
+                "ms_per_step": r["e2e_ms"],
+                "api": "hardkv_decode_step_host" if args.path == "fused" else
+                       "pinned-host copies in, the standalone calls, the output copied out"},
         "roofline": {"bound": "hbm", "kernel": KERNEL_OF_STAGE[dom], "achieved": achieved,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
                      "traffic": traffic, "alg_bytes_per_launch": by[dom],
@@ -638,7 +741,7 @@ def main(argv=None):
                   "the graph launch (events around the replay call)",
         "ms_per_step_with_graph_launch": r["outer_ms"],
         "stages_us": {s: round(v_ * 1e3, 2) for s, v_ in r["stages"].items()},
-        "stage_alg_bytes": {s: int(by[s]) for s in STAGES},
+        "stage_alg_bytes": {s: int(by[s]) for s in stages},
         "gpu_launches": r["kernels_per_step"] * args.steps * N,
         "clocks": r["clocks"],
         "device_status": [int(x) for x in r["status"]],

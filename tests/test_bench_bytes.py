@@ -15,7 +15,8 @@ element size, a row = one K row + one V row):
             step, gathered only under Sparse Loading, read once when carried over), the
             index, Dense and Condensed rows, Condensed weights, q and the fp32 output
 
-on random states of several shapes, and on one hand-worked unit.
+on random states of several shapes, and on one hand-worked unit; and the same for the
+step as its standalone calls (bench --path unfused).
 """
 import math
 
@@ -100,6 +101,53 @@ def test_one_hand_worked_unit():
     assert got["attend"] == (2 * 3637 * 512 + 3637 * 4 + (257 + 256) * 512 + 256 * 4
                              + 4 * 256 + 4 * 512)                 # 4 005 588
     assert got["total"] == 1024 + 2064384 + 63456 + 4005588      # 6 134 452
+
+
+def _by_units_unfused(w, st):
+    """The standalone calls, unit by unit: the selection writes only the mask; the
+    compaction reads the mask, writes the Cap-long index and, under Rewrite Cache, reads
+    the kept rows from the ring and writes them compact; the attention reads every kept
+    row once."""
+    e = 2 if w.dtype == synth.BF16 else 4
+    d, G, C, cap = w.head_dim, w.group, w.condensed_slots, w.sparse_cap
+    row = 2 * d * e
+    tot = dict(append=0, condense=0, select=0, regularize=0, attend=0)
+    for b in range(w.batch):
+        L = int(st["d_lo"][b] - st["s_lo"][b])
+        dense = int(st["len"][b] - st["d_lo"][b])
+        sel = bool(st["reselect"][b])
+        for h in range(w.n_kv_heads):
+            n, live = int(st["n_kept"][b, h]), int(st["live"][b, h])
+            rewrite = bool(st["sp_mode"][b, h])
+            tot["append"] += 4 * d * e
+            if w.condense_mode == synth.MERGE and st["moved"][b]:
+                tot["condense"] += (w.block + 2 * C) * row
+            words = 4 * math.ceil(L / 32)
+            if sel:
+                tot["select"] += L * d * e + G * d * e + 4 * L + 4 * L + words
+                tot["regularize"] += words + 4 * cap + (2 * n * row if rewrite else 0)
+                kept = n * row
+            else:
+                kept = live * row
+            tot["attend"] += (kept + 4 * n + (dense + C) * row + 4 * C
+                              + G * d * e + G * d * 4)
+    tot["total"] = sum(tot.values())
+    return tot
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("shape", ["bf16_merge", "f32_evict"])
+def test_unfused_bytes_match_the_per_unit_statement(shape, seed):
+    kw = {"bf16_merge": dict(condense_mode=synth.MERGE),
+          "f32_evict": dict(dtype=synth.F32, head_dim=64, n_q_heads=4, n_kv_heads=2)}[shape]
+    w = synth.small(sparse_cap=700, **kw)
+    st = _state(w, np.random.RandomState(100 + seed))
+    got = bench.step_bytes(w, st, fused=False)
+    for k, v in _by_units_unfused(w, st).items():
+        assert got[k] == v, (k, got[k], v)
+    # the fused step moves less: the kept rows are gathered once for both the rewrite and
+    # the attention, and the index is written once
+    assert bench.step_bytes(w, st)["total"] <= got["total"]
 
 
 def test_sum_bytes_pools_the_kept_fraction_over_steps():
